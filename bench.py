@@ -1,0 +1,440 @@
+#!/usr/bin/env python3
+"""Benchmark of the attention hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One JSON line on stdout (rank 0).  Two timed phases, each of exactly K steps
+after W warm-up steps, bracketed by a barrier and a device synchronisation on
+both sides, timed with CUDA events on the launching stream, max over ranks:
+
+* prefill (headline ``value``): the 70B-shaped causal GQA workload
+  (b1 S8192 H64 Hkv8 D128, RoPE theta 1e4 with linear factor 2.0, bf16).  One
+  step = RoPE table from position ids + llama_attn_prefill (K rotation pass +
+  tcgen05 attention kernel).  Throughput counts only unmasked FLOPs:
+  4 * D * (S(S+1)/2) * b * H per step.
+* decode: the GQA decode workload (b32 H64 Hkv8 D128, cache lengths uniform
+  in [512, 4096], max 4096).  One step = RoPE row for the query positions +
+  llama_attn_decode (split-KV kernel + combine).  Bytes = K and V rows read,
+  2 * sum(len_b) * Hkv * D * 2.
+
+Inputs are larger than L2 (126 MB) in both phases (prefill: q 134 MB, out
+134 MB; decode: two alternating 537 MB caches, ~302 MB read per step), so no
+L2 flush is needed between steps.  Multi-GPU runs are independent replicas
+(the path has no cross-GPU exchange): ``value`` is the sum over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+from llama_gqa_causal_b200 import workloads as W  # noqa: E402
+
+PREFILL = W.LLAMA70B
+DECODE = W.DECODE70B
+METRIC = "causal GQA prefill TFLOP/s and KV-decode HBM GB/s, % of B200 roofline"
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        d = json.load(open(p))
+        return float(d["bf16_tflops"]), float(d["bf16_tflops_sustained"]), float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return 1590.0, 1400.0, 6650.0, "fallback"
+
+
+# ----------------------------------------------------------------------------- distributed plumbing
+
+def _dist_init():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    if ws <= 1:
+        return 0, 1, 0
+    import datetime
+    import torch.distributed as dist
+    rank = int(os.environ["RANK"])
+    local = int(os.environ.get("LOCAL_RANK", rank))
+    torch.cuda.set_device(local)
+    dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                            device_id=torch.device("cuda", local))
+    return rank, ws, local
+
+
+def _barrier(ws):
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def _max_over_ranks(x: float, ws: int) -> float:
+    if ws <= 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ----------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clock and throttle reasons during a timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        out = {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        if not self.path or not os.path.exists(self.path):
+            return out
+        rows = []
+        for line in open(self.path):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                rows.append((float(f[1]), float(f[2]), f[5], f[6], f[7], f[8]))
+            except ValueError:
+                continue
+        os.unlink(self.path)
+        if not rows:
+            return out
+        out["samples"] = len(rows)
+        out["sm_mhz"] = statistics.median(r[0] for r in rows)
+        out["sm_max_mhz"] = max(r[1] for r in rows)
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        reasons = set()
+        for r in rows:
+            for n, v in zip(names, r[2:]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        out["reasons"] = sorted(reasons)
+        return out
+
+
+# ----------------------------------------------------------------------------- our arm
+
+def run_ours(args, rank, ws, local):
+    from llama_gqa_causal_b200 import api
+    api.load()
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream()
+    peak_burst, peak_sus, hbm, peak_src = _peaks()
+
+    # ------------------------------------------------------------------ prefill phase
+    cfg = PREFILL
+    x = W.prefill_inputs(cfg)
+    q, k, v = (x[n].to(dev) for n in ("q", "k", "v"))
+    pos = x["pos"].to(dev)
+    out = torch.empty(cfg.bsz, cfg.seq, cfg.n_heads * cfg.head_dim, device=dev, dtype=cfg.dtype)
+    wsp = torch.empty(api.prefill_workspace_bytes(cfg.bsz, cfg.n_heads, cfg.n_kv_heads, cfg.seq,
+                                                  cfg.head_dim, cfg.dtype, True),
+                      device=dev, dtype=torch.uint8)
+
+    def prefill_step(ev=None):
+        cos, sin = api.rope_table(pos, cfg.head_dim, cfg.theta, cfg.factor)
+        if ev is not None:
+            ev[0].record(stream)
+        api.prefill(q, k, v, cos, sin, causal=True, scale=cfg.scale, out=out, workspace=wsp)
+        if ev is not None:
+            ev[1].record(stream)
+
+    for _ in range(args.warmup):
+        prefill_step()
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        _barrier(ws)
+        torch.cuda.synchronize()
+        t0.record(stream)
+        for i in range(args.steps):
+            prefill_step(evs[i])
+        t1.record(stream)
+        torch.cuda.synchronize()
+        _barrier(ws)
+    clocks = clk.summary()
+    ms_total = _max_over_ranks(t0.elapsed_time(t1), ws)
+    ms_call = _max_over_ranks(statistics.mean(a.elapsed_time(b) for a, b in evs), ws)
+    flops = cfg.flops()
+    value = ws * flops * args.steps / (ms_total * 1e-3) / 1e12
+    achieved = flops / (ms_call * 1e-3) / 1e12
+    assert api.device_status() == api.LLAMA_OK
+
+    # e2e: pinned host inputs -> device, compute, result -> pinned host, every step
+    hq, hk, hv = (x[n].pin_memory() for n in ("q", "k", "v"))
+    hpos = x["pos"].pin_memory()
+    hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+
+    def e2e_step():
+        q.copy_(hq, non_blocking=True)
+        k.copy_(hk, non_blocking=True)
+        v.copy_(hv, non_blocking=True)
+        pos.copy_(hpos, non_blocking=True)
+        cos, sin = api.rope_table(pos, cfg.head_dim, cfg.theta, cfg.factor)
+        api.prefill(q, k, v, cos, sin, causal=True, scale=cfg.scale, out=out, workspace=wsp)
+        hout.copy_(out, non_blocking=True)
+
+    e2e_steps = max(1, min(args.steps, 5))
+    e2e_step()
+    torch.cuda.synchronize()
+    _barrier(ws)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    _barrier(ws)
+    ms_e2e = _max_over_ranks(e0.elapsed_time(e1), ws)
+    e2e_value = ws * flops * e2e_steps / (ms_e2e * 1e-3) / 1e12
+    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hpos))
+    d2h = hout.numel() * hout.element_size()
+    del hq, hk, hv, hout, q, k, v, out, wsp, x
+    torch.cuda.empty_cache()
+
+    # ------------------------------------------------------------------ decode phase
+    dcfg = DECODE
+    insts = []
+    for rep in range(2):  # two caches, alternated, so no step reads L2-resident data
+        y = W.decode_inputs(dcfg)
+        insts.append({n: y[n].to(dev) for n in ("q", "k_cache", "v_cache", "lens", "qpos")})
+    lens_cpu = y["lens"].to(torch.int64)
+    dbytes = int(2 * lens_cpu.sum().item() * dcfg.n_kv_heads * dcfg.head_dim * 2)
+    dout = torch.empty(dcfg.bsz, dcfg.n_heads * dcfg.head_dim, device=dev, dtype=dcfg.dtype)
+    dws = torch.empty(api.decode_workspace_bytes(dcfg.bsz, dcfg.n_heads, dcfg.max_cache_len,
+                                                 dcfg.head_dim), device=dev, dtype=torch.uint8)
+
+    def decode_step(i, ev=None):
+        d = insts[i % 2]
+        cos, sin = api.rope_table(d["qpos"].view(-1, 1), dcfg.head_dim, dcfg.theta, dcfg.factor)
+        if ev is not None:
+            ev[0].record(stream)
+        api.decode(d["q"], d["k_cache"], d["v_cache"], d["lens"], cos.view(dcfg.bsz, -1),
+                   sin.view(dcfg.bsz, -1), scale=dcfg.scale, out=dout, workspace=dws)
+        if ev is not None:
+            ev[1].record(stream)
+
+    dsteps = max(args.steps, 20)
+    for i in range(max(args.warmup, 3)):
+        decode_step(i)
+    torch.cuda.synchronize()
+    devs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+            for _ in range(dsteps)]
+    _barrier(ws)
+    torch.cuda.synchronize()
+    d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    d0.record(stream)
+    for i in range(dsteps):
+        decode_step(i, devs[i])
+    d1.record(stream)
+    torch.cuda.synchronize()
+    _barrier(ws)
+    ms_dec_total = _max_over_ranks(d0.elapsed_time(d1), ws)
+    ms_dec_call = _max_over_ranks(statistics.mean(a.elapsed_time(b) for a, b in devs), ws)
+    dec_value = ws * dbytes * dsteps / (ms_dec_total * 1e-3) / 1e9
+    dec_achieved = dbytes / (ms_dec_call * 1e-3) / 1e9
+    assert api.device_status() == api.LLAMA_OK
+
+    # prefill step: rope_table + K rotation + attention + decode step: rope_table + decode + combine
+    launches = args.steps * 3 + dsteps * 3
+
+    line = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": "TFLOP/s",
+        "n_gpus": ws,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_total / args.steps, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) q/k/v, cast to bf16)",
+        "config": {
+            "workload": "llama70b causal GQA prefill b1 S8192 H64 Hkv8 D128, RoPE theta 1e4 "
+                        "linear x2 (value); decode70b GQA decode b32 H64 Hkv8 D128 lens U[512,4096] "
+                        "(decode)",
+            "global_batch": cfg.bsz * ws,
+            "seq_len": cfg.seq,
+            "parallelism": f"replicas x{ws}",
+            "l2": "inputs larger than L2 (no flush)",
+        },
+        "roofline": {
+            "bound": "tensor",
+            "kernel": "llama_attn_prefill (K rotation pass + prefill_sm100_kernel)",
+            "achieved": round(achieved, 2),
+            "peak": peak_burst,
+            "unit": "TFLOP/s",
+            "frac": round(achieved / peak_burst, 4),
+            "peak_source": f"{peak_src} bf16 burst",
+            "traffic": None,
+        },
+        "decode": {
+            "value": round(dec_value, 1),
+            "unit": "GB/s",
+            "ms_per_step": round(ms_dec_total / dsteps, 4),
+            "steps": dsteps,
+            "bytes_per_step": dbytes,
+            "roofline": {
+                "bound": "hbm",
+                "kernel": "llama_attn_decode (decode_bf16_kernel + decode_combine_kernel)",
+                "achieved": round(dec_achieved, 1),
+                "peak": hbm,
+                "unit": "GB/s",
+                "frac": round(dec_achieved / hbm, 4),
+                "peak_source": f"{peak_src} copy bandwidth",
+                "traffic": None,
+            },
+        },
+        "e2e": {
+            "value": round(e2e_value, 3),
+            "unit": "TFLOP/s",
+            "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h,
+            "steps": e2e_steps,
+        },
+        "gpu_launches": launches,
+        "clocks": clocks,
+    }
+    if rank == 0 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline()
+    return line
+
+
+# ----------------------------------------------------------------------------- oracle arms
+
+def _oracle_sample_prefill(cfg, rows):
+    """Run the fp64 oracle on all heads of `rows` (lo, hi) of the workload; returns (seconds, flops)."""
+    import oracle
+    x = W.prefill_inputs(cfg)
+    lo, hi = rows
+    t = time.perf_counter()
+    oracle.prefill(x["q"], x["k"], x["v"], x["pos"], theta=cfg.theta, factor=cfg.factor,
+                   scale=cfg.scale, causal=cfg.causal, rows=rows)
+    dt = time.perf_counter() - t
+    keys = sum(min(cfg.seq, i + 1) if cfg.causal else cfg.seq for i in range(lo, hi))
+    flops = 4 * cfg.head_dim * keys * cfg.bsz * cfg.n_heads
+    return dt, flops
+
+
+def cpu_baseline(rows=None):
+    import oracle
+    cfg = PREFILL
+    rows = rows or (cfg.seq - 16, cfg.seq)
+    dt, flops = _oracle_sample_prefill(cfg, rows)
+    return {"value": round(flops / dt / 1e12, 6), "unit": "TFLOP/s", "cores": oracle.max_threads(),
+            "kind": "oracle",
+            "sample": f"llama70b prefill, all 64 heads, query rows [{rows[0]}, {rows[1]}) "
+                      f"({flops / 1e9:.1f} GFLOP fp64, {dt:.1f} s, includes rotating all K)"}
+
+
+def run_reference(args, rank, ws):
+    if rank != 0:
+        return None
+    import oracle
+    cfg = PREFILL
+    rows = (cfg.seq - 4, cfg.seq)
+    times, flops = [], 0
+    for i in range(args.warmup + args.steps):
+        dt, fl = _oracle_sample_prefill(cfg, rows)
+        if i >= args.warmup:
+            times.append(dt)
+            flops = fl
+    total = sum(times)
+    value = flops * len(times) / total / 1e12
+    return {
+        "impl": "reference",
+        "metric": METRIC,
+        "value": round(value, 6),
+        "unit": "TFLOP/s",
+        "n_gpus": 1,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(total / len(times) * 1e3, 2),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f64",
+        "data": "synthetic (seeded N(0,1) q/k/v, cast to bf16)",
+        "config": {"workload": "llama70b causal GQA prefill b1 S8192 H64 Hkv8 D128, RoPE theta 1e4 "
+                               "linear x2 (bounded sample per step)",
+                   "global_batch": 1, "seq_len": cfg.seq, "parallelism": "cpu"},
+        "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": oracle.max_threads(),
+                         "kind": "oracle",
+                         "sample": f"all 64 heads, query rows [{rows[0]}, {rows[1]}) per step"},
+        "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        rank = int(os.environ.get("RANK", "0"))
+        line = run_reference(args, rank, int(os.environ.get("WORLD_SIZE", "1")))
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return
+    rank, ws, local = _dist_init()
+    try:
+        line = run_ours(args, rank, ws, local)
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+    finally:
+        if ws > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

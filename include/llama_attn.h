@@ -1,0 +1,144 @@
+/*
+ * llama_attn.h -- C ABI of libllama_attn.so: LLaMA-style self-attention on one
+ * B200 GPU (sm_100a), prefill over a full sequence and single-token decode
+ * against a KV cache.
+ *
+ * The operation (cited by page title and section):
+ *   "[HuggingFace Transformers] LlamaAttention source walkthrough"
+ *   (blog.csdn.net), section 1.2 steps 2-5 and section 2 forward() steps 2-6:
+ *     out_h = softmax(scale * Q'_h K'_{kv(h)}^T + mask) V_{kv(h)},
+ *     heads concatenated in order 0..H-1 on the last dimension,
+ *   where Q' and K' are Q and K rotated by RoPE (step 3, rotate-half form
+ *   x*cos + rotate_half(x)*sin, rotate_half(x) = [-x[D/2:], x[:D/2]]), and
+ *   kv(h) = h / (n_heads / n_kv_heads) is the repeat_kv head map of step 4
+ *   ("Llama2 Transformer architecture and optimisation practice" (lpqz.cn),
+ *   section 2.1: query heads share one K/V head per group).  The softmax is
+ *   computed in fp32 (step 5.2).  Decode is the "KV cache" case of
+ *   "LLaMA2 large language model architecture analysis"
+ *   (obsidian-quartz-blog), section "KV cache": one query row per sequence
+ *   attends to every cached key; nothing is masked.
+ *
+ * Conventions shared by every entry point:
+ *   - All tensor pointers are DEVICE pointers, contiguous, row-major, owned by
+ *     the caller, and must be 16-byte aligned.  The library never allocates
+ *     device memory and never frees what it is given.
+ *   - All work is enqueued on `cuda_stream` (a cudaStream_t; NULL = legacy
+ *     default stream) and the call returns without synchronising.
+ *   - `dtype` (llama_dtype) applies to q, k, v, the caches and out together.
+ *     LLAMA_DT_BF16 runs the tensor-core kernels (tcgen05 prefill, mma decode)
+ *     with fp32 accumulation and an fp32 softmax; the probabilities are
+ *     rounded to bf16 before the P.V product.  LLAMA_DT_F32 runs the fp32
+ *     CUDA-core kernels (no TF32 anywhere).
+ *   - Return value is an llama_status.  Arguments are checked on the host
+ *     before anything is enqueued; on a non-zero status nothing was launched
+ *     unless the status is LLAMA_ERR_CUDA (launch failure).
+ *   - Device-side waits are bounded: a kernel whose pipeline wait runs out
+ *     (about 2 s) records LLAMA_ERR_DEVICE_TIMEOUT in a device status word and
+ *     returns; llama_attn_device_status() reads and clears it.
+ */
+#ifndef LLAMA_ATTN_H
+#define LLAMA_ATTN_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum { LLAMA_DT_F32 = 0, LLAMA_DT_BF16 = 1 } llama_dtype;
+
+typedef enum {
+  LLAMA_OK = 0,
+  LLAMA_ERR_INVALID_ARG = 1,   /* null pointer, bad size, divisibility, misalignment */
+  LLAMA_ERR_UNSUPPORTED = 2,   /* valid request this build has no kernel for (head_dim) */
+  LLAMA_ERR_CUDA = 3,          /* a CUDA runtime/driver call or launch failed */
+  LLAMA_ERR_DEVICE_TIMEOUT = 4 /* a kernel's bounded wait ran out (see above) */
+} llama_status;
+
+/*
+ * RoPE cos/sin tables ("[HuggingFace Transformers] LlamaAttention source
+ * walkthrough", section 2 step 3: cos, sin = rotary_emb(x, position_ids), from
+ * rope_theta; linear scaling from "Llama2 Transformer architecture and
+ * optimisation practice", section 6.1).
+ *   pos      device int64 [bsz * seq] position ids
+ *   cos, sin device fp32 [bsz * seq, head_dim] outputs.  For i < head_dim/2:
+ *            angle = (pos / pos_scale_factor) * theta^(-2i/head_dim), computed
+ *            in fp64 and stored as fp32 in columns i and i + head_dim/2.
+ * Errors: INVALID_ARG for null pointers, bsz/seq < 1, odd or non-positive
+ * head_dim, theta <= 0, pos_scale_factor <= 0.
+ */
+int llama_rope_table(const long long* pos, int bsz, int seq, int head_dim, double theta,
+                     double pos_scale_factor, float* cos, float* sin, void* cuda_stream);
+
+/* Device bytes of workspace llama_attn_prefill needs for this shape (0 when
+ * no RoPE or dtype is fp32).  has_rope: whether cos/sin will be passed. */
+size_t llama_attn_prefill_workspace_bytes(int bsz, int n_heads, int n_kv_heads, int seq,
+                                          int head_dim, int dtype, int has_rope);
+
+/*
+ * Full-sequence (prefill) attention.
+ *   q        [bsz, seq, n_heads, head_dim]      (projection output viewed per
+ *   k, v     [bsz, seq, n_kv_heads, head_dim]    head, no transpose: step 2)
+ *   cos, sin fp32 [bsz, seq, head_dim] or both NULL for no RoPE.  Applied to q
+ *            and k (never v) as x*cos + rotate_half(x)*sin, elementwise.
+ *   scale    multiplies q.k (usually 1/sqrt(head_dim), step 5.1)
+ *   causal   non-zero: query i sees keys j <= i (sequence index)
+ *   out      [bsz, seq, n_heads * head_dim], head h at columns [h*D, (h+1)*D)
+ *   add_mask fp32 [bsz, 1, seq, seq] or NULL; added to scale*q.k (step 5.1),
+ *            on top of `causal` when both are given.  A row whose keys are all
+ *            masked (-inf) yields zeros.
+ *   workspace / workspace_bytes: caller-owned device scratch of at least
+ *            llama_attn_prefill_workspace_bytes(...) bytes (may be NULL if 0).
+ * Errors: INVALID_ARG for null required pointers, bsz/seq/heads < 1,
+ * n_heads % n_kv_heads != 0, odd head_dim, exactly one of cos/sin NULL,
+ * non-finite scale, misaligned pointers, too small a workspace, unknown
+ * dtype; UNSUPPORTED for head_dim not in {64, 128}; CUDA for launch errors.
+ */
+int llama_attn_prefill(const void* q, const void* k, const void* v, const float* cos,
+                       const float* sin, int bsz, int n_heads, int n_kv_heads, int seq,
+                       int head_dim, float scale, int causal, void* out,
+                       const float* add_mask, int dtype, void* workspace,
+                       size_t workspace_bytes, void* cuda_stream);
+
+/* Device bytes of workspace llama_attn_decode needs (split-KV partial results). */
+size_t llama_attn_decode_workspace_bytes(int bsz, int n_heads, int max_cache_len, int head_dim);
+
+/*
+ * Single-token decode against a KV cache.
+ *   q          [bsz, n_heads, head_dim], NOT rotated: the kernel rotates it with
+ *              cos/sin (the row at the query's position)
+ *   k_cache    [bsz, n_kv_heads, max_cache_len, head_dim], keys already rotated
+ *   v_cache    [bsz, n_kv_heads, max_cache_len, head_dim]
+ *   cache_lens device int32 [bsz]: rows [0, cache_lens[b]) are attended.  Values
+ *              are clamped to [0, max_cache_len] on the device; a length of 0
+ *              yields a zero output row.  Rows at or past the length are never
+ *              read into the result (they may hold anything, NaN included).
+ *   cos, sin   fp32 [bsz, head_dim] or both NULL (no RoPE on q)
+ *   out        [bsz, n_heads * head_dim]
+ *   workspace  caller-owned device scratch of at least
+ *              llama_attn_decode_workspace_bytes(...) bytes
+ * Errors: as llama_attn_prefill, plus INVALID_ARG for max_cache_len < 1 or a
+ * NULL cache_lens.
+ */
+int llama_attn_decode(const void* q, const void* k_cache, const void* v_cache,
+                      const int* cache_lens, const float* cos, const float* sin, int bsz,
+                      int n_heads, int n_kv_heads, int max_cache_len, int head_dim,
+                      float scale, void* out, void* workspace, size_t workspace_bytes,
+                      int dtype, void* cuda_stream);
+
+/* Synchronises `cuda_stream`, then reads and clears the device status word of
+ * the current device.  Returns LLAMA_OK, LLAMA_ERR_DEVICE_TIMEOUT, or
+ * LLAMA_ERR_CUDA if the synchronisation itself failed. */
+int llama_attn_device_status(void* cuda_stream);
+
+/* Static, NUL-terminated description of a status code. */
+const char* llama_attn_status_string(int status);
+
+/* ABI version (major * 100 + minor). */
+int llama_attn_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LLAMA_ATTN_H */

@@ -1,0 +1,189 @@
+"""ctypes binding of libllama_attn.so: the same entry points, torch tensors in.
+
+Argument marshalling only: tensors become device pointers, the current torch
+CUDA stream becomes ``cuda_stream``, outputs and workspaces are allocated by
+torch when the caller does not pass them, and a non-zero status raises.  Every
+step of the computation runs in the library's kernels.  There is no CPU
+fallback: without the built library, or on a tensor that is not on a CUDA
+device, the call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from typing import Optional, Tuple
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libllama_attn.so")
+
+LLAMA_DT_F32 = 0
+LLAMA_DT_BF16 = 1
+LLAMA_OK = 0
+LLAMA_ERR_INVALID_ARG = 1
+LLAMA_ERR_UNSUPPORTED = 2
+LLAMA_ERR_CUDA = 3
+LLAMA_ERR_DEVICE_TIMEOUT = 4
+
+# Every symbol include/llama_attn.h declares.
+EXPORTED = (
+    "llama_rope_table",
+    "llama_attn_prefill_workspace_bytes",
+    "llama_attn_prefill",
+    "llama_attn_decode_workspace_bytes",
+    "llama_attn_decode",
+    "llama_attn_device_status",
+    "llama_attn_status_string",
+    "llama_attn_abi_version",
+)
+
+_lib = None
+
+
+class LlamaAttnError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)} (status {status})")
+
+
+def load() -> ctypes.CDLL:
+    """Load the in-tree library (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(
+            f"{LIB_PATH} is missing: build it with `python -m llama_gqa_causal_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    P, I, D, Z, F = ctypes.c_void_p, ctypes.c_int, ctypes.c_double, ctypes.c_size_t, ctypes.c_float
+    lib.llama_rope_table.argtypes = [P, I, I, I, D, D, P, P, P]
+    lib.llama_rope_table.restype = I
+    lib.llama_attn_prefill_workspace_bytes.argtypes = [I, I, I, I, I, I, I]
+    lib.llama_attn_prefill_workspace_bytes.restype = Z
+    lib.llama_attn_prefill.argtypes = [P, P, P, P, P, I, I, I, I, I, F, I, P, P, I, P, Z, P]
+    lib.llama_attn_prefill.restype = I
+    lib.llama_attn_decode_workspace_bytes.argtypes = [I, I, I, I]
+    lib.llama_attn_decode_workspace_bytes.restype = Z
+    lib.llama_attn_decode.argtypes = [P, P, P, P, P, P, I, I, I, I, I, F, P, P, Z, I, P]
+    lib.llama_attn_decode.restype = I
+    lib.llama_attn_device_status.argtypes = [P]
+    lib.llama_attn_device_status.restype = I
+    lib.llama_attn_status_string.argtypes = [I]
+    lib.llama_attn_status_string.restype = ctypes.c_char_p
+    lib.llama_attn_abi_version.argtypes = []
+    lib.llama_attn_abi_version.restype = I
+    _lib = lib
+    return lib
+
+
+def status_string(status: int) -> str:
+    return load().llama_attn_status_string(int(status)).decode()
+
+
+def _check(status: int, where: str) -> None:
+    if status != LLAMA_OK:
+        raise LlamaAttnError(status, where)
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("llama_attn: tensors must live on a CUDA device")
+    if not t.is_contiguous():
+        raise ValueError("llama_attn: tensors must be contiguous")
+    return t.data_ptr()
+
+
+def _stream(stream=None) -> int:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return s.cuda_stream
+
+
+def _dtype_code(dt: torch.dtype) -> int:
+    if dt == torch.bfloat16:
+        return LLAMA_DT_BF16
+    if dt == torch.float32:
+        return LLAMA_DT_F32
+    raise ValueError(f"llama_attn: unsupported dtype {dt}")
+
+
+def rope_table(pos: torch.Tensor, head_dim: int, theta: float = 10000.0,
+               factor: float = 1.0, stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """cos, sin [*pos.shape, head_dim] fp32 from int64 positions (llama_rope_table)."""
+    lib = load()
+    pos = pos.to(torch.int64).contiguous()
+    n = pos.numel()
+    cos = torch.empty(*pos.shape, head_dim, device=pos.device, dtype=torch.float32)
+    sin = torch.empty_like(cos)
+    bsz = pos.shape[0] if pos.dim() > 1 else 1
+    seq = n // bsz
+    _check(lib.llama_rope_table(_ptr(pos), bsz, seq, head_dim, float(theta), float(factor),
+                                _ptr(cos), _ptr(sin), _stream(stream)), "llama_rope_table")
+    return cos, sin
+
+
+def prefill_workspace_bytes(bsz, n_heads, n_kv_heads, seq, head_dim, dtype, has_rope) -> int:
+    return int(load().llama_attn_prefill_workspace_bytes(
+        bsz, n_heads, n_kv_heads, seq, head_dim, _dtype_code(dtype), int(bool(has_rope))))
+
+
+def decode_workspace_bytes(bsz, n_heads, max_cache_len, head_dim) -> int:
+    return int(load().llama_attn_decode_workspace_bytes(bsz, n_heads, max_cache_len, head_dim))
+
+
+def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+            cos: Optional[torch.Tensor] = None, sin: Optional[torch.Tensor] = None, *,
+            causal: bool = True, scale: Optional[float] = None,
+            mask: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None,
+            workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """llama_attn_prefill.  q [b,S,H,D], k/v [b,S,Hkv,D] -> out [b, S, H*D]."""
+    lib = load()
+    b, S, H, D = q.shape
+    Hkv = k.shape[2]
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    if out is None:
+        out = torch.empty(b, S, H * D, device=q.device, dtype=q.dtype)
+    need = prefill_workspace_bytes(b, H, Hkv, S, D, q.dtype, cos is not None)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, device=q.device, dtype=torch.uint8)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib.llama_attn_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(cos), _ptr(sin), b, H, Hkv, S,
+                                  D, float(scale), int(bool(causal)), _ptr(out), _ptr(mask),
+                                  _dtype_code(q.dtype), _ptr(workspace), ws_bytes,
+                                  _stream(stream)), "llama_attn_prefill")
+    return out
+
+
+def decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+           cache_lens: torch.Tensor, cos: Optional[torch.Tensor] = None,
+           sin: Optional[torch.Tensor] = None, *, scale: Optional[float] = None,
+           out: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+           stream=None) -> torch.Tensor:
+    """llama_attn_decode.  q [b,H,D], caches [b,Hkv,L,D], cache_lens int32 [b] -> out [b, H*D]."""
+    lib = load()
+    b, H, D = q.shape
+    Hkv, L = k_cache.shape[1], k_cache.shape[2]
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    if out is None:
+        out = torch.empty(b, H * D, device=q.device, dtype=q.dtype)
+    if workspace is None:
+        workspace = torch.empty(decode_workspace_bytes(b, H, L, D), device=q.device,
+                                dtype=torch.uint8)
+    ws_bytes = workspace.numel() * workspace.element_size()
+    if cache_lens.dtype != torch.int32:
+        raise ValueError("llama_attn_decode: cache_lens must be int32")
+    _check(lib.llama_attn_decode(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(cache_lens),
+                                 _ptr(cos), _ptr(sin), b, H, Hkv, L, D, float(scale), _ptr(out),
+                                 _ptr(workspace), ws_bytes, _dtype_code(q.dtype),
+                                 _stream(stream)), "llama_attn_decode")
+    return out
+
+
+def device_status(stream=None) -> int:
+    """llama_attn_device_status: sync the stream, read and clear the device status word."""
+    return int(load().llama_attn_device_status(_stream(stream)))

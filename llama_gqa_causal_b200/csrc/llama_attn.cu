@@ -1,0 +1,330 @@
+// C ABI of libllama_attn.so (declared in include/llama_attn.h): argument
+// validation, TMA tensor-map encoding and kernel dispatch.  Every kernel of
+// the library is compiled into this one translation unit.
+#include <math.h>
+#include <stdint.h>
+#include <stdio.h>
+
+#include <algorithm>
+#include <mutex>
+
+#include "llama_attn.h"
+
+#include "common.cuh"
+#include "attn_fp32.cuh"
+#include "decode_bf16.cuh"
+#include "prefill_sm100.cuh"
+#include "rope.cuh"
+
+namespace {
+
+constexpr int kAbiVersion = 100;
+constexpr int kDecodeSplitRows = 512;  // cache rows per decode CTA (multiple of dec::TR)
+
+// ---------------------------------------------------------------- host helpers
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  });
+  return fn;
+}
+
+// bf16 tensor map with the 128-byte swizzle; dims/strides innermost first
+// (strides in bytes, for dims 1..rank-1), box innermost first.
+bool make_map(CUtensorMap* m, const void* base, int rank, const cuuint64_t* dims,
+              const cuuint64_t* strides, const cuuint32_t* box) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, static_cast<cuuint32_t>(rank),
+                  const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// Dynamic shared memory opt-in, once per (kernel, device).
+template <typename K>
+bool ensure_smem_attr(K kernel, size_t bytes) {
+  static bool done[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  if (dev >= 0 && dev < 64 && done[dev]) return true;
+  cudaError_t e =
+      cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes));
+  if (e != cudaSuccess) return false;
+  if (dev >= 0 && dev < 64) done[dev] = true;
+  return true;
+}
+
+int launch_status() {
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    fprintf(stderr, "llama_attn: launch failed: %s\n", cudaGetErrorString(e));
+    return LLAMA_ERR_CUDA;
+  }
+  return LLAMA_OK;
+}
+
+int check_common(int bsz, int n_heads, int n_kv_heads, int head_dim, int dtype,
+                 const float* cos, const float* sin, float scale) {
+  if (bsz < 1 || n_heads < 1 || n_kv_heads < 1 || head_dim < 2) return LLAMA_ERR_INVALID_ARG;
+  if (n_heads % n_kv_heads != 0) return LLAMA_ERR_INVALID_ARG;
+  if (head_dim % 2 != 0) return LLAMA_ERR_INVALID_ARG;
+  if ((cos == nullptr) != (sin == nullptr)) return LLAMA_ERR_INVALID_ARG;
+  if (!isfinite(scale)) return LLAMA_ERR_INVALID_ARG;
+  if (dtype != LLAMA_DT_F32 && dtype != LLAMA_DT_BF16) return LLAMA_ERR_INVALID_ARG;
+  if (head_dim != 64 && head_dim != 128) return LLAMA_ERR_UNSUPPORTED;
+  return LLAMA_OK;
+}
+
+int decode_splits(int max_cache_len) {
+  return (max_cache_len + kDecodeSplitRows - 1) / kDecodeSplitRows;
+}
+
+// ---------------------------------------------------------------- prefill dispatch
+template <int D>
+int prefill_bf16(const void* q, const void* k, const void* v, const float* cos, const float* sin,
+                 int bsz, int H, int Hkv, int S, float scale, int causal, void* out,
+                 const float* mask, void* workspace, cudaStream_t st) {
+  const void* k_src = k;
+  if (cos != nullptr) {  // rotate every K row once into the workspace
+    const long long n_tok = static_cast<long long>(bsz) * S;
+    const long long work = n_tok * Hkv * (D / 16);
+    const int threads = 256;
+    const int blocks = static_cast<int>(std::min<long long>((work + threads - 1) / threads, 148LL * 16));
+    la::rope_rotate_bf16_kernel<D><<<blocks, threads, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(k), static_cast<__nv_bfloat16*>(workspace), cos, sin,
+        n_tok, Hkv);
+    if (int e = launch_status()) return e;
+    k_src = workspace;
+  }
+  CUtensorMap tk, tv;
+  const cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(Hkv),
+                              static_cast<cuuint64_t>(S), static_cast<cuuint64_t>(bsz)};
+  const cuuint64_t strides[3] = {static_cast<cuuint64_t>(D) * 2,
+                                 static_cast<cuuint64_t>(Hkv) * D * 2,
+                                 static_cast<cuuint64_t>(S) * Hkv * D * 2};
+  const cuuint32_t box[4] = {64, 1, static_cast<cuuint32_t>(la::pf::BN), 1};
+  if (!make_map(&tk, k_src, 4, dims, strides, box)) return LLAMA_ERR_CUDA;
+  if (!make_map(&tv, v, 4, dims, strides, box)) return LLAMA_ERR_CUDA;
+
+  la::PrefillParams p;
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.cos = cos;
+  p.sin = sin;
+  p.mask = mask;
+  p.out = static_cast<__nv_bfloat16*>(out);
+  p.bsz = bsz;
+  p.H = H;
+  p.Hkv = Hkv;
+  p.S = S;
+  p.group = H / Hkv;
+  p.n_pb = (S + la::pf::BM - 1) / la::pf::BM;
+  p.n_kb = (S + la::pf::BN - 1) / la::pf::BN;
+  p.ctas_per_kvh = (p.group * p.n_pb + la::pf::NQ - 1) / la::pf::NQ;
+  p.causal = causal ? 1 : 0;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  const size_t smem = sizeof(la::PfSmem<D>) + 1024;
+  if (!ensure_smem_attr(la::prefill_sm100_kernel<D>, smem)) return LLAMA_ERR_CUDA;
+  const long long grid = static_cast<long long>(bsz) * Hkv * p.ctas_per_kvh;
+  if (grid > 0x7fffffffLL) return LLAMA_ERR_INVALID_ARG;
+  la::prefill_sm100_kernel<D><<<static_cast<unsigned>(grid), la::pf::THREADS, smem, st>>>(tk, tv, p);
+  return launch_status();
+}
+
+template <int D>
+int attn_fp32(const float* q, const float* k, const float* v, const float* cos, const float* sin,
+              const float* mask, const int* lens, float* out, int bsz, int H, int Hkv, int S,
+              int L, int decode, int causal, float scale, cudaStream_t st) {
+  la::Fp32Params p;
+  p.q = q; p.k = k; p.v = v; p.cos = cos; p.sin = sin; p.mask = mask; p.lens = lens; p.out = out;
+  p.bsz = bsz; p.H = H; p.Hkv = Hkv; p.S = S; p.L = L; p.group = H / Hkv;
+  p.decode = decode; p.causal = causal ? 1 : 0; p.scale = scale;
+  dim3 grid;
+  if (!decode) grid = dim3((S + 31) / 32, H, bsz);
+  else grid = dim3((p.group + 31) / 32, Hkv, bsz);
+  la::attn_fp32_kernel<D><<<grid, 128, 0, st>>>(p);
+  return launch_status();
+}
+
+template <int D>
+int decode_bf16(const void* q, const void* kc, const void* vc, const int* lens, const float* cos,
+                const float* sin, int bsz, int H, int Hkv, int L, float scale, void* out,
+                void* workspace, cudaStream_t st) {
+  const int n_splits = decode_splits(L);
+  CUtensorMap tk, tv;
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(L),
+                              static_cast<cuuint64_t>(bsz) * Hkv};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(L) * D * 2};
+  const cuuint32_t box[3] = {64, static_cast<cuuint32_t>(la::dec::TR), 1};
+  if (!make_map(&tk, kc, 3, dims, strides, box)) return LLAMA_ERR_CUDA;
+  if (!make_map(&tv, vc, 3, dims, strides, box)) return LLAMA_ERR_CUDA;
+  la::DecodeParams p;
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.cos = cos;
+  p.sin = sin;
+  p.lens = lens;
+  p.ws_o = static_cast<float*>(workspace);
+  p.ws_ml = p.ws_o + static_cast<size_t>(bsz) * H * n_splits * D;
+  p.bsz = bsz;
+  p.H = H;
+  p.Hkv = Hkv;
+  p.L = L;
+  p.group = H / Hkv;
+  p.hchunks = (p.group + 7) / 8;
+  p.split_rows = kDecodeSplitRows;
+  p.n_splits = n_splits;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  const size_t smem = sizeof(la::DecSmem<D>) + 1024;
+  if (!ensure_smem_attr(la::decode_bf16_kernel<D>, smem)) return LLAMA_ERR_CUDA;
+  dim3 grid(n_splits, Hkv * p.hchunks, bsz);
+  la::decode_bf16_kernel<D><<<grid, la::dec::THREADS, smem, st>>>(tk, tv, p);
+  if (int e = launch_status()) return e;
+  la::decode_combine_kernel<D><<<dim3(H, bsz), D, 0, st>>>(
+      p.ws_o, p.ws_ml, lens, static_cast<__nv_bfloat16*>(out), H, L, kDecodeSplitRows, n_splits);
+  return launch_status();
+}
+
+}  // namespace
+
+extern "C" {
+
+int llama_attn_abi_version(void) { return kAbiVersion; }
+
+const char* llama_attn_status_string(int status) {
+  switch (status) {
+    case LLAMA_OK: return "ok";
+    case LLAMA_ERR_INVALID_ARG: return "invalid argument";
+    case LLAMA_ERR_UNSUPPORTED: return "unsupported configuration";
+    case LLAMA_ERR_CUDA: return "CUDA error";
+    case LLAMA_ERR_DEVICE_TIMEOUT: return "device-side wait timed out";
+    default: return "unknown status";
+  }
+}
+
+int llama_rope_table(const long long* pos, int bsz, int seq, int head_dim, double theta,
+                     double pos_scale_factor, float* cos, float* sin, void* cuda_stream) {
+  if (!pos || !cos || !sin) return LLAMA_ERR_INVALID_ARG;
+  if (bsz < 1 || seq < 1 || head_dim < 2 || (head_dim % 2)) return LLAMA_ERR_INVALID_ARG;
+  if (!(theta > 0.0) || !(pos_scale_factor > 0.0)) return LLAMA_ERR_INVALID_ARG;
+  const long long n = static_cast<long long>(bsz) * seq;
+  const long long work = n * (head_dim / 2);
+  const int threads = 256;
+  const int blocks = static_cast<int>(std::min<long long>((work + threads - 1) / threads, 148LL * 32));
+  la::rope_table_kernel<<<blocks, threads, 0, as_stream(cuda_stream)>>>(
+      pos, n, head_dim, theta, pos_scale_factor, cos, sin);
+  return launch_status();
+}
+
+size_t llama_attn_prefill_workspace_bytes(int bsz, int n_heads, int n_kv_heads, int seq,
+                                          int head_dim, int dtype, int has_rope) {
+  (void)n_heads;
+  if (dtype != LLAMA_DT_BF16 || !has_rope || bsz < 1 || n_kv_heads < 1 || seq < 1 || head_dim < 1)
+    return 0;
+  return static_cast<size_t>(bsz) * seq * n_kv_heads * head_dim * 2;  // rotated K, bf16
+}
+
+int llama_attn_prefill(const void* q, const void* k, const void* v, const float* cos,
+                       const float* sin, int bsz, int n_heads, int n_kv_heads, int seq,
+                       int head_dim, float scale, int causal, void* out,
+                       const float* add_mask, int dtype, void* workspace,
+                       size_t workspace_bytes, void* cuda_stream) {
+  if (!q || !k || !v || !out) return LLAMA_ERR_INVALID_ARG;
+  if (seq < 1) return LLAMA_ERR_INVALID_ARG;
+  if (int e = check_common(bsz, n_heads, n_kv_heads, head_dim, dtype, cos, sin, scale)) return e;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(cos) ||
+      !aligned16(sin) || !aligned16(add_mask) || !aligned16(workspace))
+    return LLAMA_ERR_INVALID_ARG;
+  const size_t need = llama_attn_prefill_workspace_bytes(bsz, n_heads, n_kv_heads, seq, head_dim,
+                                                         dtype, cos != nullptr);
+  if (need > 0 && (workspace == nullptr || workspace_bytes < need)) return LLAMA_ERR_INVALID_ARG;
+  cudaStream_t st = as_stream(cuda_stream);
+  if (dtype == LLAMA_DT_BF16) {
+    if (head_dim == 128)
+      return prefill_bf16<128>(q, k, v, cos, sin, bsz, n_heads, n_kv_heads, seq, scale, causal,
+                               out, add_mask, workspace, st);
+    return prefill_bf16<64>(q, k, v, cos, sin, bsz, n_heads, n_kv_heads, seq, scale, causal, out,
+                            add_mask, workspace, st);
+  }
+  const float* qf = static_cast<const float*>(q);
+  const float* kf = static_cast<const float*>(k);
+  const float* vf = static_cast<const float*>(v);
+  float* of = static_cast<float*>(out);
+  if (head_dim == 128)
+    return attn_fp32<128>(qf, kf, vf, cos, sin, add_mask, nullptr, of, bsz, n_heads, n_kv_heads,
+                          seq, seq, 0, causal, scale, st);
+  return attn_fp32<64>(qf, kf, vf, cos, sin, add_mask, nullptr, of, bsz, n_heads, n_kv_heads, seq,
+                       seq, 0, causal, scale, st);
+}
+
+size_t llama_attn_decode_workspace_bytes(int bsz, int n_heads, int max_cache_len, int head_dim) {
+  if (bsz < 1 || n_heads < 1 || max_cache_len < 1 || head_dim < 1) return 0;
+  const size_t slots = static_cast<size_t>(bsz) * n_heads * decode_splits(max_cache_len);
+  return slots * (static_cast<size_t>(head_dim) + 2) * sizeof(float);
+}
+
+int llama_attn_decode(const void* q, const void* k_cache, const void* v_cache,
+                      const int* cache_lens, const float* cos, const float* sin, int bsz,
+                      int n_heads, int n_kv_heads, int max_cache_len, int head_dim,
+                      float scale, void* out, void* workspace, size_t workspace_bytes,
+                      int dtype, void* cuda_stream) {
+  if (!q || !k_cache || !v_cache || !cache_lens || !out) return LLAMA_ERR_INVALID_ARG;
+  if (max_cache_len < 1) return LLAMA_ERR_INVALID_ARG;
+  if (int e = check_common(bsz, n_heads, n_kv_heads, head_dim, dtype, cos, sin, scale)) return e;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out) ||
+      !aligned16(cos) || !aligned16(sin) || !aligned16(workspace) ||
+      (reinterpret_cast<uintptr_t>(cache_lens) & 3u))
+    return LLAMA_ERR_INVALID_ARG;
+  cudaStream_t st = as_stream(cuda_stream);
+  if (dtype == LLAMA_DT_BF16) {
+    const size_t need = llama_attn_decode_workspace_bytes(bsz, n_heads, max_cache_len, head_dim);
+    if (workspace == nullptr || workspace_bytes < need) return LLAMA_ERR_INVALID_ARG;
+    if (head_dim == 128)
+      return decode_bf16<128>(q, k_cache, v_cache, cache_lens, cos, sin, bsz, n_heads, n_kv_heads,
+                              max_cache_len, scale, out, workspace, st);
+    return decode_bf16<64>(q, k_cache, v_cache, cache_lens, cos, sin, bsz, n_heads, n_kv_heads,
+                           max_cache_len, scale, out, workspace, st);
+  }
+  const float* qf = static_cast<const float*>(q);
+  if (head_dim == 128)
+    return attn_fp32<128>(qf, static_cast<const float*>(k_cache),
+                          static_cast<const float*>(v_cache), cos, sin, nullptr, cache_lens,
+                          static_cast<float*>(out), bsz, n_heads, n_kv_heads, 1, max_cache_len, 1,
+                          0, scale, st);
+  return attn_fp32<64>(qf, static_cast<const float*>(k_cache), static_cast<const float*>(v_cache),
+                       cos, sin, nullptr, cache_lens, static_cast<float*>(out), bsz, n_heads,
+                       n_kv_heads, 1, max_cache_len, 1, 0, scale, st);
+}
+
+int llama_attn_device_status(void* cuda_stream) {
+  if (cudaStreamSynchronize(as_stream(cuda_stream)) != cudaSuccess) return LLAMA_ERR_CUDA;
+  unsigned int word = 0;
+  if (cudaMemcpyFromSymbol(&word, la::g_device_status, sizeof(word)) != cudaSuccess)
+    return LLAMA_ERR_CUDA;
+  if (word != 0) {
+    const unsigned int zero = 0;
+    if (cudaMemcpyToSymbol(la::g_device_status, &zero, sizeof(zero)) != cudaSuccess)
+      return LLAMA_ERR_CUDA;
+    return LLAMA_ERR_DEVICE_TIMEOUT;
+  }
+  return LLAMA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,385 @@
+// bf16 prefill attention on the 5th-generation tensor cores (tcgen05 + TMEM + TMA).
+//
+// Computes, for each query head h and query position i,
+//   out[b, i, h*D:(h+1)*D] = softmax_j(scale * q'_i . k'_j + mask_ij) v_j
+// ("[HuggingFace Transformers] LlamaAttention source walkthrough", section
+// 1.2 steps 2-4 and section 2 steps 3-6), with j <= i when causal, K/V head
+// h / group (repeat_kv, step 4), fp32 scores and softmax (step 5.2) and the
+// probabilities rounded to bf16 before the product with V (the `.to(dtype)`
+// of step 5.2).
+//
+// Work unit: a Q tile = 128 consecutive query positions of one query head.
+// The Q tiles of one (batch, K/V head) are ordered position-block-major, so
+// consecutive units are the heads of one GQA group at the same positions (or,
+// with group 1, consecutive position blocks).  A CTA owns two consecutive
+// units and streams each K/V tile of 128 keys through shared memory once for
+// both; causal tiles past a unit's last position are skipped.
+//
+// Warp roles (384 threads):
+//   warp 0      TMA producer: K' and V tiles (2 stages each), 128B swizzle
+//   warp 1      TMEM allocator and MMA issuer (one thread):
+//                 S_t = Q_t K_j^T   (SS: both operands K-major in smem)
+//                 O_t += P_t V_j    (TS: P from TMEM, V MN-major in smem)
+//   warps 4-7   softmax of unit 0, warps 8-11 softmax of unit 1: each thread
+//               owns one query row (= one TMEM lane).  Before the loop they
+//               rotate their Q row with RoPE and write it to shared memory
+//               (this is the "RoPE while staging Q" step); K arrives already
+//               rotated (a separate pass rotates each K row exactly once).
+// TMEM (512 columns): S_0, S_1 (128 fp32 columns each), O_0, O_1 (D each).
+// P_t (bf16, two per column) is written over the first 64 columns of S_t:
+// the MMA warp issues the next S_t = Q_t K^T only after O_t += P_t V in the
+// same tcgen05 issue order, so the overwrite follows the read.
+// Rescaling of O is lazy: the running max used for the exponentials moves
+// only when a row's max grows by more than 2^8, which keeps O corrections rare.
+#pragma once
+#include "common.cuh"
+
+namespace la {
+namespace pf {
+constexpr int BM = 128;       // query rows per tile (= TMEM lanes)
+constexpr int BN = 128;       // keys per K/V tile
+constexpr int NQ = 2;         // Q tiles (units) per CTA
+constexpr int KSTAGES = 2;
+constexpr int VSTAGES = 2;
+constexpr int THREADS = 384;
+constexpr float kRescaleThreshold = 8.0f;  // log2 units
+}  // namespace pf
+
+struct PrefillParams {
+  const __nv_bfloat16* q;  // [b, S, H, D]
+  const float* cos;        // [b, S, D] or null
+  const float* sin;
+  const float* mask;       // [b, 1, S, S] or null
+  __nv_bfloat16* out;      // [b, S, H*D]
+  int bsz, H, Hkv, S, group;
+  int n_pb;                // ceil(S / BM)
+  int n_kb;                // ceil(S / BN)
+  int ctas_per_kvh;        // ceil(group * n_pb / 2)
+  int causal;
+  float scale_log2;        // scale * log2(e)
+};
+
+template <int D>
+struct PfSmem {
+  alignas(1024) __nv_bfloat16 q[pf::NQ][pf::BM * D];
+  alignas(1024) __nv_bfloat16 k[pf::KSTAGES][pf::BN * D];
+  alignas(1024) __nv_bfloat16 v[pf::VSTAGES][pf::BN * D];
+  uint64_t k_full[pf::KSTAGES], k_empty[pf::KSTAGES];
+  uint64_t v_full[pf::VSTAGES], v_empty[pf::VSTAGES];
+  uint64_t q_ready[pf::NQ], s_full[pf::NQ], p_full[pf::NQ], o_full[pf::NQ];
+  uint64_t mma_done;
+  uint32_t tmem_base;
+};
+
+template <int D>
+__global__ void __launch_bounds__(pf::THREADS, 1)
+    prefill_sm100_kernel(const __grid_constant__ CUtensorMap tm_k,
+                         const __grid_constant__ CUtensorMap tm_v, PrefillParams p) {
+  using namespace pf;
+  constexpr int CB = D / 64;                       // 64-column swizzle blocks per row
+  constexpr uint32_t BLOCK_BYTES = BM * 128;       // one [128 rows x 64 cols] bf16 block
+  constexpr uint32_t TILE_BYTES = BM * D * 2;
+  constexpr uint32_t IDESC_QK = idesc_bf16(BM, BN, false);
+  constexpr uint32_t IDESC_PV = idesc_bf16(BM, D, true);
+  constexpr uint32_t TMEM_COLS = 512;
+
+  extern __shared__ uint8_t smem_raw[];
+  PfSmem<D>& s = *reinterpret_cast<PfSmem<D>*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  // ---- work decomposition: heavy (late position blocks) CTAs first
+  const int n_bkv = p.bsz * p.Hkv;
+  const int rank = blockIdx.x / n_bkv;
+  const int bkv = blockIdx.x - rank * n_bkv;
+  const int b = bkv / p.Hkv, kvh = bkv - (bkv / p.Hkv) * p.Hkv;
+  const int cta = p.ctas_per_kvh - 1 - rank;
+  const int n_units = p.group * p.n_pb;
+  int unit_pb[NQ], unit_head[NQ], unit_nkv[NQ];
+#pragma unroll
+  for (int t = 0; t < NQ; ++t) {
+    const int u = cta * NQ + t;
+    if (u < n_units) {
+      unit_pb[t] = u / p.group;
+      unit_head[t] = kvh * p.group + (u - unit_pb[t] * p.group);
+      unit_nkv[t] = p.causal ? min(p.n_kb, ((unit_pb[t] + 1) * BM + BN - 1) / BN) : p.n_kb;
+    } else {
+      unit_pb[t] = 0;
+      unit_head[t] = 0;
+      unit_nkv[t] = 0;
+    }
+  }
+  const int n_max = max(unit_nkv[0], unit_nkv[1]);
+
+  // ---- setup
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < KSTAGES; ++i) { mbar_init(&s.k_full[i], 1); mbar_init(&s.k_empty[i], 1); }
+    for (int i = 0; i < VSTAGES; ++i) { mbar_init(&s.v_full[i], 1); mbar_init(&s.v_empty[i], 1); }
+    for (int t = 0; t < NQ; ++t) {
+      mbar_init(&s.q_ready[t], 128);
+      mbar_init(&s.s_full[t], 1);
+      mbar_init(&s.p_full[t], 128);
+      mbar_init(&s.o_full[t], 1);
+    }
+    mbar_init(&s.mma_done, 1);
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&s.tmem_base, TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = s.tmem_base;
+  const uint32_t tm_s[NQ] = {tmem, tmem + BN};
+  const uint32_t tm_o[NQ] = {tmem + 2 * BN, tmem + 2 * BN + D};
+
+  if (warp == 0) {
+    // ================================================================ TMA producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      int k_issued = 0, v_issued = 0;
+      for (int j = 0; j < n_max; ++j) {
+        const int ks = j % KSTAGES;
+        if (j >= KSTAGES && !mbar_wait(&s.k_empty[ks], ((j / KSTAGES) - 1) & 1)) break;
+        mbar_arrive_expect_tx(&s.k_full[ks], TILE_BYTES);
+#pragma unroll
+        for (int cb = 0; cb < CB; ++cb)
+          tma_load_4d(reinterpret_cast<uint8_t*>(&s.k[ks][0]) + cb * BLOCK_BYTES, &tm_k,
+                      &s.k_full[ks], cb * 64, kvh, j * BN, b);
+        k_issued = j + 1;
+        const int vs = j % VSTAGES;
+        if (j >= VSTAGES && !mbar_wait(&s.v_empty[vs], ((j / VSTAGES) - 1) & 1)) break;
+        mbar_arrive_expect_tx(&s.v_full[vs], TILE_BYTES);
+#pragma unroll
+        for (int cb = 0; cb < CB; ++cb)
+          tma_load_4d(reinterpret_cast<uint8_t*>(&s.v[vs][0]) + cb * BLOCK_BYTES, &tm_v,
+                      &s.v_full[vs], cb * 64, kvh, j * BN, b);
+        v_issued = j + 1;
+      }
+      // leave no copy in flight
+      for (int j = max(0, k_issued - KSTAGES); j < k_issued; ++j)
+        if (!mbar_wait(&s.k_full[j % KSTAGES], (j / KSTAGES) & 1)) break;
+      for (int j = max(0, v_issued - VSTAGES); j < v_issued; ++j)
+        if (!mbar_wait(&s.v_full[j % VSTAGES], (j / VSTAGES) & 1)) break;
+    }
+  } else if (warp == 1) {
+    // ================================================================ MMA issuer
+    if (lane == 0) {
+      bool ok = true;
+      const uint32_t q_addr[NQ] = {smem_u32(&s.q[0][0]), smem_u32(&s.q[1][0])};
+      auto issue_qk = [&](int t, int ks) {
+        const uint32_t ka = smem_u32(&s.k[ks][0]);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk / 4) * BLOCK_BYTES + (kk % 4) * 32;
+          mma_ss(tm_s[t], sw128_desc(q_addr[t] + off, 16, 1024), sw128_desc(ka + off, 16, 1024),
+                 IDESC_QK, kk > 0 ? 1u : 0u);
+        }
+      };
+      auto issue_pv = [&](int t, int vs, bool accumulate) {
+        const uint32_t va = smem_u32(&s.v[vs][0]);
+#pragma unroll
+        for (int kk = 0; kk < BN / 16; ++kk) {
+          // A = P_t[:, 16kk:16kk+16] in TMEM (8 columns of packed bf16 pairs);
+          // B = V rows 16kk.. (MN-major: 64-dim blocks BLOCK_BYTES apart, 8-row groups 1 KB apart)
+          mma_ts(tm_o[t], tm_s[t] + kk * 8, sw128_desc(va + kk * 2048, BLOCK_BYTES, 1024),
+                 IDESC_PV, (accumulate || kk > 0) ? 1u : 0u);
+        }
+      };
+      for (int t = 0; t < NQ && ok; ++t)
+        if (unit_nkv[t] > 0) ok = mbar_wait(&s.q_ready[t], 0);
+      if (ok && n_max > 0) ok = mbar_wait(&s.k_full[0], 0);
+      if (ok && n_max > 0) {
+        tc_fence_after();
+        for (int t = 0; t < NQ; ++t)
+          if (unit_nkv[t] > 0) {
+            issue_qk(t, 0);
+            tc_commit(&s.s_full[t]);
+          }
+        tc_commit(&s.k_empty[0]);
+      }
+      for (int j = 0; j < n_max && ok; ++j) {
+        const int vs = j % VSTAGES;
+        if (!mbar_wait(&s.v_full[vs], (j / VSTAGES) & 1)) { ok = false; break; }
+        const int jn = j + 1;
+        const bool next = jn < n_max;
+        if (next && !mbar_wait(&s.k_full[jn % KSTAGES], (jn / KSTAGES) & 1)) { ok = false; break; }
+        for (int t = 0; t < NQ; ++t) {
+          if (j >= unit_nkv[t]) continue;
+          if (!mbar_wait(&s.p_full[t], j & 1)) { ok = false; break; }
+          tc_fence_after();
+          issue_pv(t, vs, j > 0);
+          if (jn == unit_nkv[t]) {
+            tc_commit(&s.o_full[t]);
+          } else {
+            issue_qk(t, jn % KSTAGES);
+            tc_commit(&s.s_full[t]);
+          }
+        }
+        if (!ok) break;
+        tc_commit(&s.v_empty[vs]);
+        if (next) tc_commit(&s.k_empty[jn % KSTAGES]);
+      }
+      // every MMA this thread issued has completed before the CTA can exit
+      tc_commit(&s.mma_done);
+      mbar_wait(&s.mma_done, 0);
+    }
+  } else if (warp >= 4) {
+    // ================================================================ softmax / epilogue
+    const int t = (warp - 4) >> 2;     // unit handled by this warpgroup
+    const int quarter = warp & 3;      // TMEM lane quarter of this warp
+    const int r = quarter * 32 + lane; // row of the Q tile = TMEM lane
+    const int n_kv = unit_nkv[t];
+    if (n_kv > 0) {
+      const int head = unit_head[t];
+      const int i = unit_pb[t] * BM + r;  // query position (sequence index)
+      const bool row_valid = i < p.S;
+      // ---- stage Q: rotate this row and write it swizzled into s.q[t]
+      {
+        uint8_t* qs = reinterpret_cast<uint8_t*>(&s.q[t][0]);
+        const __nv_bfloat16* qr = p.q + ((static_cast<size_t>(b) * p.S + i) * p.H + head) * D;
+        const float* cr = p.cos ? p.cos + (static_cast<size_t>(b) * p.S + i) * D : nullptr;
+        const float* sr = p.sin ? p.sin + (static_cast<size_t>(b) * p.S + i) * D : nullptr;
+#pragma unroll
+        for (int c = 0; c < D / 16; ++c) {  // chunk c of the first half, c + D/16 of the second
+          uint4 lo = make_uint4(0, 0, 0, 0), hi = make_uint4(0, 0, 0, 0);
+          if (row_valid) {
+            const uint4 a = *reinterpret_cast<const uint4*>(qr + c * 8);
+            const uint4 z = *reinterpret_cast<const uint4*>(qr + D / 2 + c * 8);
+            if (cr) {
+              const uint32_t au[4] = {a.x, a.y, a.z, a.w}, zu[4] = {z.x, z.y, z.z, z.w};
+              uint32_t lu[4], hu[4];
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const int d = c * 8 + 2 * e;
+                const float x0 = bf16lo(au[e]), x1 = bf16hi(au[e]);
+                const float z0 = bf16lo(zu[e]), z1 = bf16hi(zu[e]);
+                lu[e] = pack_bf16x2(fmaf(x0, cr[d], -z0 * sr[d]), fmaf(x1, cr[d + 1], -z1 * sr[d + 1]));
+                hu[e] = pack_bf16x2(fmaf(z0, cr[d + D / 2], x0 * sr[d + D / 2]),
+                                    fmaf(z1, cr[d + D / 2 + 1], x1 * sr[d + D / 2 + 1]));
+              }
+              lo = make_uint4(lu[0], lu[1], lu[2], lu[3]);
+              hi = make_uint4(hu[0], hu[1], hu[2], hu[3]);
+            } else {
+              lo = a;
+              hi = z;
+            }
+          }
+          const int c2 = c + D / 16;
+          *reinterpret_cast<uint4*>(qs + (c / 8) * BLOCK_BYTES + sw128_offset(r, c % 8)) = lo;
+          *reinterpret_cast<uint4*>(qs + (c2 / 8) * BLOCK_BYTES + sw128_offset(r, c2 % 8)) = hi;
+        }
+        fence_proxy_async_smem();
+        mbar_arrive(&s.q_ready[t]);
+      }
+
+      const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+      const float* mrow = p.mask ? p.mask + (static_cast<size_t>(b) * p.S + i) * p.S : nullptr;
+      float m_ref = -INFINITY;  // reference max (log2 units) of the exponentials
+      float l_sum = 0.f;
+      bool ok = true;
+      for (int j = 0; j < n_kv; ++j) {
+        if (!mbar_wait(&s.s_full[t], j & 1)) { ok = false; break; }
+        tc_fence_after();
+        uint32_t sr[4][32];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tmem_ld32(tm_s[t] + lane_off + c * 32, sr[c]);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tmem_ld_wait(sr[c]);
+        float x[BN];
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+#pragma unroll
+          for (int e = 0; e < 32; ++e) x[c * 32 + e] = __uint_as_float(sr[c][e]) * p.scale_log2;
+        const int key0 = j * BN;
+        const bool edge = (key0 + BN > p.S) || (p.causal && key0 + BN - 1 > unit_pb[t] * BM) ||
+                          (mrow != nullptr);
+        if (edge) {
+          const int lim = p.causal ? min(p.S - 1, i) : p.S - 1;  // last visible key
+#pragma unroll
+          for (int e = 0; e < BN; ++e) {
+            const int key = key0 + e;
+            float xv = x[e];
+            if (mrow != nullptr && key < p.S) xv = fmaf(mrow[key], 1.4426950408889634f, xv);
+            x[e] = (key <= lim) ? xv : -INFINITY;
+          }
+        }
+        float mx = x[0];
+#pragma unroll
+        for (int e = 1; e < BN; ++e) mx = fmaxf(mx, x[e]);
+        // lazy reference: move only when the max grows by more than the threshold
+        float alpha = 1.f;
+        if (mx > m_ref + kRescaleThreshold || (m_ref == -INFINITY && mx != -INFINITY)) {
+          alpha = (m_ref == -INFINITY) ? 0.f : ex2_approx(m_ref - mx);
+          m_ref = mx;
+        }
+        const float mref_use = (m_ref == -INFINITY) ? 0.f : m_ref;
+        uint32_t pk[2][32];
+        float rs = 0.f;
+#pragma unroll
+        for (int e = 0; e < BN; e += 2) {
+          const float p0 = ex2_approx(x[e] - mref_use);
+          const float p1 = ex2_approx(x[e + 1] - mref_use);
+          rs += p0 + p1;
+          pk[e / 64][(e % 64) / 2] = pack_bf16x2(p0, p1);
+        }
+        l_sum = fmaf(l_sum, alpha, rs);
+        // O correction (warp-collective TMEM access when any row of the warp needs it)
+        if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t orr[32];
+            tmem_ld32(tm_o[t] + lane_off + c * 32, orr);
+            tmem_ld_wait(orr);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) orr[e] = __float_as_uint(__uint_as_float(orr[e]) * alpha);
+            tmem_st32(tm_o[t] + lane_off + c * 32, orr);
+          }
+        }
+        tmem_st32(tm_s[t] + lane_off, pk[0]);
+        tmem_st32(tm_s[t] + lane_off + 32, pk[1]);
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(&s.p_full[t]);
+      }
+      // ---- epilogue: O / l -> bf16 -> out[b, i, head*D : head*D + D]
+      if (ok && mbar_wait(&s.o_full[t], 0)) {
+        tc_fence_after();
+        const float inv = (l_sum > 0.f) ? 1.f / l_sum : 0.f;
+        __nv_bfloat16* orow = p.out + (static_cast<size_t>(b) * p.S + i) * (static_cast<size_t>(p.H) * D) +
+                              static_cast<size_t>(head) * D;
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t orr[32];
+          tmem_ld32(tm_o[t] + lane_off + c * 32, orr);
+          tmem_ld_wait(orr);
+          if (row_valid) {
+#pragma unroll
+            for (int e = 0; e < 32; e += 8) {
+              uint4 w;
+              w.x = pack_bf16x2(__uint_as_float(orr[e]) * inv, __uint_as_float(orr[e + 1]) * inv);
+              w.y = pack_bf16x2(__uint_as_float(orr[e + 2]) * inv, __uint_as_float(orr[e + 3]) * inv);
+              w.z = pack_bf16x2(__uint_as_float(orr[e + 4]) * inv, __uint_as_float(orr[e + 5]) * inv);
+              w.w = pack_bf16x2(__uint_as_float(orr[e + 6]) * inv, __uint_as_float(orr[e + 7]) * inv);
+              *reinterpret_cast<uint4*>(orow + c * 32 + e) = w;
+            }
+          }
+        }
+      }
+    }
+  }
+
+  // ---- teardown
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+}  // namespace la

@@ -1,0 +1,144 @@
+"""Host-side checks of the C ABI: the library loads, exports every declared
+symbol, and rejects bad arguments before anything is enqueued.
+
+No test here launches a kernel: every call below carries an argument the
+library must refuse on the host, so the same tests are safe on a GPU machine.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+from llama_gqa_causal_b200 import api, build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "llama_attn.h")
+
+FAKE = 0x10000  # a 16-byte aligned non-null address; never dereferenced (calls are rejected first)
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return api.load()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(llama_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_binding_symbols():
+    assert declared_functions() == sorted(api.EXPORTED)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+        assert isinstance(getattr(lib, name), ctypes._CFuncPtr)
+
+
+def test_abi_version_and_status_strings(lib):
+    assert lib.llama_attn_abi_version() == 100
+    assert api.status_string(0) == "ok"
+    assert "invalid" in api.status_string(1)
+    assert "unsupported" in api.status_string(2)
+    assert "CUDA" in api.status_string(3)
+    assert "timed out" in api.status_string(4)
+    assert api.status_string(99) == "unknown status"
+
+
+def test_workspace_sizes(lib):
+    # prefill: rotated K in bf16 when RoPE is on, nothing otherwise / for fp32
+    assert lib.llama_attn_prefill_workspace_bytes(1, 64, 8, 8192, 128, 1, 1) == 8192 * 8 * 128 * 2
+    assert lib.llama_attn_prefill_workspace_bytes(1, 64, 8, 8192, 128, 1, 0) == 0
+    assert lib.llama_attn_prefill_workspace_bytes(1, 4, 2, 64, 64, 0, 1) == 0
+    # decode: (D + 2) floats per (b, head, split of 512 rows)
+    assert lib.llama_attn_decode_workspace_bytes(32, 64, 4096, 128) == 32 * 64 * 8 * 130 * 4
+    assert lib.llama_attn_decode_workspace_bytes(2, 4, 513, 64) == 2 * 4 * 2 * 66 * 4
+    assert lib.llama_attn_decode_workspace_bytes(0, 4, 513, 64) == 0
+
+
+def _prefill(lib, **kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, cos=None, sin=None, bsz=1, H=4, Hkv=2, S=64, D=64,
+             scale=0.125, causal=1, out=FAKE, mask=None, dtype=1, ws=None, ws_bytes=0, stream=None)
+    a.update(kw)
+    return lib.llama_attn_prefill(a["q"], a["k"], a["v"], a["cos"], a["sin"], a["bsz"], a["H"],
+                                  a["Hkv"], a["S"], a["D"], a["scale"], a["causal"], a["out"],
+                                  a["mask"], a["dtype"], a["ws"], a["ws_bytes"], a["stream"])
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(q=None), 1),
+    (dict(out=None), 1),
+    (dict(v=None), 1),
+    (dict(bsz=0), 1),
+    (dict(S=0), 1),
+    (dict(H=0), 1),
+    (dict(H=6, Hkv=4), 1),            # n_heads % n_kv_heads != 0 (divisibility, as TP demands)
+    (dict(D=63), 1),                  # odd head_dim: rotate-half needs pairs
+    (dict(cos=FAKE), 1),              # cos without sin
+    (dict(scale=float("nan")), 1),
+    (dict(scale=float("inf")), 1),
+    (dict(dtype=7), 1),
+    (dict(q=FAKE + 8), 1),            # misaligned
+    (dict(mask=FAKE + 4), 1),
+    (dict(cos=FAKE, sin=FAKE, ws=None, ws_bytes=0), 1),        # RoPE needs the K workspace
+    (dict(cos=FAKE, sin=FAKE, ws=FAKE, ws_bytes=64 * 2 * 64), 1),  # too small by half
+    (dict(D=96), 2),                  # valid but no kernel for this head_dim
+    (dict(D=256), 2),
+])
+def test_prefill_rejects(lib, kw, status):
+    assert _prefill(lib, **kw) == status
+
+
+def _decode(lib, **kw):
+    a = dict(q=FAKE, kc=FAKE, vc=FAKE, lens=FAKE, cos=None, sin=None, bsz=2, H=8, Hkv=2, L=100,
+             D=128, scale=0.1, out=FAKE, ws=FAKE, ws_bytes=1 << 30, dtype=1, stream=None)
+    a.update(kw)
+    return lib.llama_attn_decode(a["q"], a["kc"], a["vc"], a["lens"], a["cos"], a["sin"], a["bsz"],
+                                 a["H"], a["Hkv"], a["L"], a["D"], a["scale"], a["out"], a["ws"],
+                                 a["ws_bytes"], a["dtype"], a["stream"])
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(lens=None), 1),
+    (dict(kc=None), 1),
+    (dict(L=0), 1),
+    (dict(H=8, Hkv=3), 1),
+    (dict(D=7), 1),
+    (dict(sin=FAKE), 1),
+    (dict(ws=None), 1),
+    (dict(ws_bytes=100), 1),
+    (dict(lens=FAKE + 2), 1),
+    (dict(vc=FAKE + 4), 1),
+    (dict(dtype=-1), 1),
+    (dict(D=80), 2),
+])
+def test_decode_rejects(lib, kw, status):
+    assert _decode(lib, **kw) == status
+
+
+@pytest.mark.parametrize("args", [
+    (None, 1, 4, 64, 1e4, 1.0, FAKE, FAKE),
+    (FAKE, 0, 4, 64, 1e4, 1.0, FAKE, FAKE),
+    (FAKE, 1, 4, 63, 1e4, 1.0, FAKE, FAKE),
+    (FAKE, 1, 4, 64, 0.0, 1.0, FAKE, FAKE),
+    (FAKE, 1, 4, 64, 1e4, -2.0, FAKE, FAKE),
+    (FAKE, 1, 4, 64, 1e4, 1.0, None, FAKE),
+])
+def test_rope_table_rejects(lib, args):
+    assert lib.llama_rope_table(*args, None) == 1
+
+
+def test_python_binding_refuses_cpu_tensors(lib):
+    import torch
+    q = torch.zeros(1, 4, 2, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        api.prefill(q, q[:, :, :1], q[:, :, :1], causal=True)
+
+
+def test_build_flags_target_sm100a():
+    assert "arch=compute_100a,code=sm_100a" in " ".join(build.FLAGS)
