@@ -38,7 +38,7 @@ sys.path.insert(0, ROOT)
 
 import torch  # noqa: E402
 
-from llama_gqa_causal_b200 import workloads as W  # noqa: E402
+from llama_gqa_causal_b200 import replicas, workloads as W  # noqa: E402
 
 PREFILL = W.LLAMA70B
 DECODE = W.DECODE70B
@@ -56,33 +56,12 @@ def _peaks():
 
 # ----------------------------------------------------------------------------- distributed plumbing
 
-def _dist_init():
-    ws = int(os.environ.get("WORLD_SIZE", "1"))
-    if ws <= 1:
-        return 0, 1, 0
-    import datetime
-    import torch.distributed as dist
-    rank = int(os.environ["RANK"])
-    local = int(os.environ.get("LOCAL_RANK", rank))
-    torch.cuda.set_device(local)
-    dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                            device_id=torch.device("cuda", local))
-    return rank, ws, local
-
-
 def _barrier(ws):
-    if ws > 1:
-        import torch.distributed as dist
-        dist.barrier()
+    replicas.barrier(ws)
 
 
 def _max_over_ranks(x: float, ws: int) -> float:
-    if ws <= 1:
-        return x
-    import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
-    dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    return float(t.item())
+    return replicas.max_over_ranks(x, ws, device="cuda")
 
 
 # ----------------------------------------------------------------------------- clocks
@@ -159,7 +138,31 @@ def run_ours(args, rank, ws, local):
     stream = torch.cuda.current_stream()
     peak_burst, peak_sus, hbm, peak_src = _peaks()
 
-    # ------------------------------------------------------------------ prefill phase
+    line = {
+        "metric": METRIC,
+        "n_gpus": ws,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) q/k/v, cast to bf16)",
+    }
+    launches = 0
+    if args.phase in ("all", "prefill"):
+        launches += _prefill_phase(args, ws, local, dev, stream, line)
+    if args.phase in ("all", "decode"):
+        launches += _decode_phase(args, ws, local, dev, stream, line)
+    line["gpu_launches"] = launches
+    if rank == 0 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline()
+    return line
+
+
+def _prefill_phase(args, ws, local, dev, stream, line):
+    from llama_gqa_causal_b200 import api
+    peak_burst, peak_sus, hbm, peak_src = _peaks()
     cfg = PREFILL
     x = W.prefill_inputs(cfg)
     q, k, v = (x[n].to(dev) for n in ("q", "k", "v"))
@@ -196,7 +199,7 @@ def run_ours(args, rank, ws, local):
     ms_total = _max_over_ranks(t0.elapsed_time(t1), ws)
     ms_call = _max_over_ranks(statistics.mean(a.elapsed_time(b) for a, b in evs), ws)
     flops = cfg.flops()
-    value = ws * flops * args.steps / (ms_total * 1e-3) / 1e12
+    value = replicas.job_throughput(flops, args.steps, ms_total, ws) / 1e12
     achieved = flops / (ms_call * 1e-3) / 1e12
     assert api.device_status() == api.LLAMA_OK
 
@@ -214,8 +217,11 @@ def run_ours(args, rank, ws, local):
         api.prefill(q, k, v, cos, sin, causal=True, scale=cfg.scale, out=out, workspace=wsp)
         hout.copy_(out, non_blocking=True)
 
-    e2e_steps = max(1, min(args.steps, 5))
-    e2e_step()
+    e2e_steps = 0 if args.no_e2e else max(1, min(args.steps, 5))
+    if e2e_steps == 0:
+        hq = hk = hv = hout = None
+    else:
+        e2e_step()
     torch.cuda.synchronize()
     _barrier(ws)
     torch.cuda.synchronize()
@@ -227,13 +233,53 @@ def run_ours(args, rank, ws, local):
     torch.cuda.synchronize()
     _barrier(ws)
     ms_e2e = _max_over_ranks(e0.elapsed_time(e1), ws)
-    e2e_value = ws * flops * e2e_steps / (ms_e2e * 1e-3) / 1e12
-    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hpos))
-    d2h = hout.numel() * hout.element_size()
+    if e2e_steps:
+        e2e_value = replicas.job_throughput(flops, e2e_steps, ms_e2e, ws) / 1e12
+        h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hpos))
+        d2h = hout.numel() * hout.element_size()
+    else:
+        e2e_value, h2d, d2h = None, 0, 0
     del hq, hk, hv, hout, q, k, v, out, wsp, x
     torch.cuda.empty_cache()
+    line.update({
+        "value": round(value, 2),
+        "unit": "TFLOP/s",
+        "ms_per_step": round(ms_total / args.steps, 4),
+        "config": {
+            "workload": "llama70b causal GQA prefill b1 S8192 H64 Hkv8 D128, RoPE theta 1e4 "
+                        "linear x2 (value); decode70b GQA decode b32 H64 Hkv8 D128 lens U[512,4096] "
+                        "(decode)",
+            "global_batch": cfg.bsz * ws,
+            "seq_len": cfg.seq,
+            "parallelism": f"replicas x{ws}",
+            "l2": "inputs larger than L2 (no flush)",
+        },
+        "roofline": {
+            "bound": "tensor",
+            "kernel": "llama_attn_prefill (K rotation pass + prefill_sm100_kernel)",
+            "achieved": round(achieved, 2),
+            "peak": peak_burst,
+            "unit": "TFLOP/s",
+            "frac": round(achieved / peak_burst, 4),
+            "peak_source": f"{peak_src} bf16 burst",
+            "traffic": None,
+        },
+        "e2e": {
+            "value": None if e2e_value is None else round(e2e_value, 3),
+            "unit": "TFLOP/s",
+            "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h,
+            "steps": e2e_steps,
+        },
+        "clocks": clocks,
+    })
+    # rope_table + K rotation + attention kernel per timed step
+    return args.steps * 3
 
-    # ------------------------------------------------------------------ decode phase
+
+def _decode_phase(args, ws, local, dev, stream, line):
+    from llama_gqa_causal_b200 import api
+    peak_burst, peak_sus, hbm, peak_src = _peaks()
     dcfg = DECODE
     insts = []
     for rep in range(2):  # two caches, alternated, so no step reads L2-resident data
@@ -272,75 +318,36 @@ def run_ours(args, rank, ws, local):
     _barrier(ws)
     ms_dec_total = _max_over_ranks(d0.elapsed_time(d1), ws)
     ms_dec_call = _max_over_ranks(statistics.mean(a.elapsed_time(b) for a, b in devs), ws)
-    dec_value = ws * dbytes * dsteps / (ms_dec_total * 1e-3) / 1e9
+    dec_value = replicas.job_throughput(dbytes, dsteps, ms_dec_total, ws) / 1e9
     dec_achieved = dbytes / (ms_dec_call * 1e-3) / 1e9
     assert api.device_status() == api.LLAMA_OK
 
-    # prefill step: rope_table + K rotation + attention + decode step: rope_table + decode + combine
-    launches = args.steps * 3 + dsteps * 3
-
-    line = {
-        "metric": METRIC,
-        "value": round(value, 2),
-        "unit": "TFLOP/s",
-        "n_gpus": ws,
-        "steps": args.steps,
-        "warmup": args.warmup,
-        "ms_per_step": round(ms_total / args.steps, 4),
-        "higher_is_better": True,
-        "scaling": "weak",
-        "vs_baseline": None,
-        "dtype": "bf16",
-        "data": "synthetic (seeded N(0,1) q/k/v, cast to bf16)",
-        "config": {
-            "workload": "llama70b causal GQA prefill b1 S8192 H64 Hkv8 D128, RoPE theta 1e4 "
-                        "linear x2 (value); decode70b GQA decode b32 H64 Hkv8 D128 lens U[512,4096] "
-                        "(decode)",
-            "global_batch": cfg.bsz * ws,
-            "seq_len": cfg.seq,
-            "parallelism": f"replicas x{ws}",
-            "l2": "inputs larger than L2 (no flush)",
-        },
+    line["decode"] = {
+        "value": round(dec_value, 1),
+        "unit": "GB/s",
+        "ms_per_step": round(ms_dec_total / dsteps, 4),
+        "steps": dsteps,
+        "bytes_per_step": dbytes,
         "roofline": {
-            "bound": "tensor",
-            "kernel": "llama_attn_prefill (K rotation pass + prefill_sm100_kernel)",
-            "achieved": round(achieved, 2),
-            "peak": peak_burst,
-            "unit": "TFLOP/s",
-            "frac": round(achieved / peak_burst, 4),
-            "peak_source": f"{peak_src} bf16 burst",
+            "bound": "hbm",
+            "kernel": "llama_attn_decode (decode_bf16_kernel + decode_combine_kernel)",
+            "achieved": round(dec_achieved, 1),
+            "peak": hbm,
+            "unit": "GB/s",
+            "frac": round(dec_achieved / hbm, 4),
+            "peak_source": f"{peak_src} copy bandwidth",
             "traffic": None,
         },
-        "decode": {
-            "value": round(dec_value, 1),
-            "unit": "GB/s",
-            "ms_per_step": round(ms_dec_total / dsteps, 4),
-            "steps": dsteps,
-            "bytes_per_step": dbytes,
-            "roofline": {
-                "bound": "hbm",
-                "kernel": "llama_attn_decode (decode_bf16_kernel + decode_combine_kernel)",
-                "achieved": round(dec_achieved, 1),
-                "peak": hbm,
-                "unit": "GB/s",
-                "frac": round(dec_achieved / hbm, 4),
-                "peak_source": f"{peak_src} copy bandwidth",
-                "traffic": None,
-            },
-        },
-        "e2e": {
-            "value": round(e2e_value, 3),
-            "unit": "TFLOP/s",
-            "h2d_bytes_per_step": h2d,
-            "d2h_bytes_per_step": d2h,
-            "steps": e2e_steps,
-        },
-        "gpu_launches": launches,
-        "clocks": clocks,
     }
-    if rank == 0 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline()
-    return line
+    if "value" not in line:  # decode-only run: the decode numbers are the line's
+        line.update({"value": line["decode"]["value"], "unit": "GB/s",
+                     "ms_per_step": line["decode"]["ms_per_step"],
+                     "config": {"workload": "decode70b GQA decode b32 H64 Hkv8 D128 lens U[512,4096]",
+                                "global_batch": dcfg.bsz * ws, "seq_len": dcfg.max_cache_len,
+                                "parallelism": f"replicas x{ws}",
+                                "l2": "two alternating caches larger than L2"}})
+    # rope_table + split kernel + combine kernel per timed step
+    return dsteps * 3
 
 
 # ----------------------------------------------------------------------------- oracle arms
@@ -416,6 +423,10 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer e2e measurement")
+    ap.add_argument("--phase", choices=["all", "prefill", "decode"], default="all",
+                    help="run only one timed phase (for profiling one kernel); the JSON "
+                         "line then carries only that phase")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -425,15 +436,13 @@ def main():
         if line is not None:
             print(json.dumps(line), flush=True)
         return
-    rank, ws, local = _dist_init()
+    rank, ws, local = replicas.init("nccl")
     try:
         line = run_ours(args, rank, ws, local)
         if rank == 0:
             print(json.dumps(line), flush=True)
     finally:
-        if ws > 1:
-            import torch.distributed as dist
-            dist.destroy_process_group()
+        replicas.shutdown(ws)
 
 
 if __name__ == "__main__":

@@ -59,9 +59,10 @@ bool make_map(CUtensorMap* m, const void* base, int rank, const cuuint64_t* dims
   return r == CUDA_SUCCESS;
 }
 
-// Dynamic shared memory opt-in, once per (kernel, device).
-template <typename K>
-bool ensure_smem_attr(K kernel, size_t bytes) {
+// Dynamic shared memory opt-in, once per (kernel, device).  Templated on the
+// kernel itself so that every instantiation keeps its own flags.
+template <auto kernel>
+bool ensure_smem_attr(size_t bytes) {
   static bool done[64] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return false;
@@ -142,7 +143,7 @@ int prefill_bf16(const void* q, const void* k, const void* v, const float* cos, 
   p.causal = causal ? 1 : 0;
   p.scale_log2 = scale * 1.4426950408889634f;
   const size_t smem = sizeof(la::PfSmem<D>) + 1024;
-  if (!ensure_smem_attr(la::prefill_sm100_kernel<D>, smem)) return LLAMA_ERR_CUDA;
+  if (!ensure_smem_attr<la::prefill_sm100_kernel<D>>(smem)) return LLAMA_ERR_CUDA;
   const long long grid = static_cast<long long>(bsz) * Hkv * p.ctas_per_kvh;
   if (grid > 0x7fffffffLL) return LLAMA_ERR_INVALID_ARG;
   la::prefill_sm100_kernel<D><<<static_cast<unsigned>(grid), la::pf::THREADS, smem, st>>>(tk, tv, p);
@@ -193,7 +194,7 @@ int decode_bf16(const void* q, const void* kc, const void* vc, const int* lens, 
   p.n_splits = n_splits;
   p.scale_log2 = scale * 1.4426950408889634f;
   const size_t smem = sizeof(la::DecSmem<D>) + 1024;
-  if (!ensure_smem_attr(la::decode_bf16_kernel<D>, smem)) return LLAMA_ERR_CUDA;
+  if (!ensure_smem_attr<la::decode_bf16_kernel<D>>(smem)) return LLAMA_ERR_CUDA;
   dim3 grid(n_splits, Hkv * p.hchunks, bsz);
   la::decode_bf16_kernel<D><<<grid, la::dec::THREADS, smem, st>>>(tk, tv, p);
   if (int e = launch_status()) return e;

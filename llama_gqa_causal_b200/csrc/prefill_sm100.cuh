@@ -15,13 +15,15 @@
 // units and streams each K/V tile of 128 keys through shared memory once for
 // both; causal tiles past a unit's last position are skipped.
 //
-// Warp roles (384 threads):
+// Warp roles (384 threads = three warpgroups):
 //   warp 0      TMA producer: K' and V tiles (2 stages each), 128B swizzle
 //   warp 1      TMEM allocator and MMA issuer (one thread):
 //                 S_t = Q_t K_j^T   (SS: both operands K-major in smem)
 //                 O_t += P_t V_j    (TS: P from TMEM, V MN-major in smem)
+//   warps 2-3   idle (complete warpgroup 0, which gives registers away)
 //   warps 4-7   softmax of unit 0, warps 8-11 softmax of unit 1: each thread
-//               owns one query row (= one TMEM lane).  Before the loop they
+//               owns one query row (= one TMEM lane; warp w reaches the 32
+//               lanes of quarter w % 4).  Before the loop they
 //               rotate their Q row with RoPE and write it to shared memory
 //               (this is the "RoPE while staging Q" step); K arrives already
 //               rotated (a separate pass rotates each K row exactly once).
@@ -41,7 +43,11 @@ constexpr int BN = 128;       // keys per K/V tile
 constexpr int NQ = 2;         // Q tiles (units) per CTA
 constexpr int KSTAGES = 2;
 constexpr int VSTAGES = 2;
-constexpr int THREADS = 384;
+constexpr int THREADS = 384;  // warpgroup 0: TMA + MMA warps; warpgroups 1, 2: softmax
+// Register budget per warpgroup after setmaxnreg: each SMSP holds one warp of
+// every warpgroup, 56 + 224 + 224 registers x 32 lanes = 16128 <= 16384.
+constexpr int kRegsControl = 56;
+constexpr int kRegsSoftmax = 224;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 }  // namespace pf
 
@@ -135,9 +141,9 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
   const uint32_t tmem = s.tmem_base;
   const uint32_t tm_s[NQ] = {tmem, tmem + BN};
   const uint32_t tm_o[NQ] = {tmem + 2 * BN, tmem + 2 * BN + D};
-
   if (warp == 0) {
     // ================================================================ TMA producer
+    setmaxnreg_dec<kRegsControl>();
     if (lane == 0) {
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
@@ -168,6 +174,7 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
     }
   } else if (warp == 1) {
     // ================================================================ MMA issuer
+    setmaxnreg_dec<kRegsControl>();
     if (lane == 0) {
       bool ok = true;
       const uint32_t q_addr[NQ] = {smem_u32(&s.q[0][0]), smem_u32(&s.q[1][0])};
@@ -228,8 +235,11 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
       tc_commit(&s.mma_done);
       mbar_wait(&s.mma_done, 0);
     }
-  } else if (warp >= 4) {
+  } else if (warp < 4) {
+    setmaxnreg_dec<kRegsControl>();  // idle warps of warpgroup 0
+  } else {
     // ================================================================ softmax / epilogue
+    setmaxnreg_inc<kRegsSoftmax>();
     const int t = (warp - 4) >> 2;     // unit handled by this warpgroup
     const int quarter = warp & 3;      // TMEM lane quarter of this warp
     const int r = quarter * 32 + lane; // row of the Q tile = TMEM lane
@@ -279,6 +289,8 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
 
       const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
       const float* mrow = p.mask ? p.mask + (static_cast<size_t>(b) * p.S + i) * p.S : nullptr;
+      const float c_log2 = p.scale_log2;
+      const bool scale_pos = c_log2 > 0.f;
       float m_ref = -INFINITY;  // reference max (log2 units) of the exponentials
       float l_sum = 0.f;
       bool ok = true;
@@ -290,43 +302,56 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
         for (int c = 0; c < 4; ++c) tmem_ld32(tm_s[t] + lane_off + c * 32, sr[c]);
 #pragma unroll
         for (int c = 0; c < 4; ++c) tmem_ld_wait(sr[c]);
-        float x[BN];
-#pragma unroll
-        for (int c = 0; c < 4; ++c)
-#pragma unroll
-          for (int e = 0; e < 32; ++e) x[c * 32 + e] = __uint_as_float(sr[c][e]) * p.scale_log2;
+        // v: raw scores (fast tiles: the scale is folded into the exponent's FMA) or
+        // scaled + masked scores (tiles that touch the diagonal, the ragged end or a mask)
+        float v[BN];
         const int key0 = j * BN;
         const bool edge = (key0 + BN > p.S) || (p.causal && key0 + BN - 1 > unit_pb[t] * BM) ||
-                          (mrow != nullptr);
-        if (edge) {
+                          (mrow != nullptr) || !scale_pos;
+        if (!edge) {
+#pragma unroll
+          for (int e = 0; e < BN; ++e) v[e] = __uint_as_float(sr[e / 32][e % 32]);
+        } else {
           const int lim = p.causal ? min(p.S - 1, i) : p.S - 1;  // last visible key
 #pragma unroll
           for (int e = 0; e < BN; ++e) {
             const int key = key0 + e;
-            float xv = x[e];
+            float xv = __uint_as_float(sr[e / 32][e % 32]) * c_log2;
             if (mrow != nullptr && key < p.S) xv = fmaf(mrow[key], 1.4426950408889634f, xv);
-            x[e] = (key <= lim) ? xv : -INFINITY;
+            v[e] = (key <= lim) ? xv : -INFINITY;
           }
         }
-        float mx = x[0];
+        // row max: eight independent 3-input chains, then a small tree
+        float mm[8];
 #pragma unroll
-        for (int e = 1; e < BN; ++e) mx = fmaxf(mx, x[e]);
+        for (int k = 0; k < 8; ++k) mm[k] = fmaxf(v[k], v[k + 8]);
+#pragma unroll
+        for (int e = 16; e < BN; e += 16)
+#pragma unroll
+          for (int k = 0; k < 8; ++k) mm[k] = fmax3f(mm[k], v[e + k], v[e + k + 8]);
+        float mx = fmax3f(fmax3f(mm[0], mm[1], mm[2]), fmax3f(mm[3], mm[4], mm[5]), fmaxf(mm[6], mm[7]));
+        if (!edge) mx *= c_log2;
         // lazy reference: move only when the max grows by more than the threshold
         float alpha = 1.f;
         if (mx > m_ref + kRescaleThreshold || (m_ref == -INFINITY && mx != -INFINITY)) {
           alpha = (m_ref == -INFINITY) ? 0.f : ex2_approx(m_ref - mx);
           m_ref = mx;
         }
-        const float mref_use = (m_ref == -INFINITY) ? 0.f : m_ref;
+        const float nref = (m_ref == -INFINITY) ? 0.f : -m_ref;
+        const float cc = edge ? 1.f : c_log2;
         uint32_t pk[2][32];
-        float rs = 0.f;
+        float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int e = 0; e < BN; e += 2) {
-          const float p0 = ex2_approx(x[e] - mref_use);
-          const float p1 = ex2_approx(x[e + 1] - mref_use);
-          rs += p0 + p1;
+          float a0, a1;
+          ffma2(a0, a1, v[e], v[e + 1], cc, cc, nref, nref);  // exponent = v*c - m_ref
+          const float p0 = ex2_approx(a0);
+          const float p1 = ex2_approx(a1);
+          const int k = (e / 2) % 4;
+          fadd2(acc[2 * k], acc[2 * k + 1], acc[2 * k], acc[2 * k + 1], p0, p1);
           pk[e / 64][(e % 64) / 2] = pack_bf16x2(p0, p1);
         }
+        const float rs = ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
         l_sum = fmaf(l_sum, alpha, rs);
         // O correction (warp-collective TMEM access when any row of the warp needs it)
         if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
