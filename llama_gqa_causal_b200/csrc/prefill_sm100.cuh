@@ -34,6 +34,8 @@
 // Rescaling of O is lazy: the running max used for the exponentials moves
 // only when a row's max grows by more than 2^8, which keeps O corrections rare.
 #pragma once
+#include <type_traits>
+
 #include "common.cuh"
 
 namespace la {
@@ -49,6 +51,12 @@ constexpr int THREADS = 384;  // warpgroup 0: TMA + MMA warps; warpgroups 1, 2: 
 constexpr int kRegsControl = 56;
 constexpr int kRegsSoftmax = 224;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
+// Of every 8 consecutive pairs of probabilities in an interior tile, this
+// many are exponentiated on the FMA pipe (exp2_poly2), the rest on MUFU.
+#ifndef LA_POLY_PAIRS_OF_8
+#define LA_POLY_PAIRS_OF_8 2
+#endif
+constexpr int kPolyPairsOf8 = LA_POLY_PAIRS_OF_8;
 }  // namespace pf
 
 struct PrefillParams {
@@ -101,22 +109,18 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
   const int bkv = blockIdx.x - rank * n_bkv;
   const int b = bkv / p.Hkv, kvh = bkv - (bkv / p.Hkv) * p.Hkv;
   const int cta = p.ctas_per_kvh - 1 - rank;
+  // two units per CTA, kept in scalars (never in arrays indexed at run time)
   const int n_units = p.group * p.n_pb;
-  int unit_pb[NQ], unit_head[NQ], unit_nkv[NQ];
-#pragma unroll
-  for (int t = 0; t < NQ; ++t) {
-    const int u = cta * NQ + t;
-    if (u < n_units) {
-      unit_pb[t] = u / p.group;
-      unit_head[t] = kvh * p.group + (u - unit_pb[t] * p.group);
-      unit_nkv[t] = p.causal ? min(p.n_kb, ((unit_pb[t] + 1) * BM + BN - 1) / BN) : p.n_kb;
-    } else {
-      unit_pb[t] = 0;
-      unit_head[t] = 0;
-      unit_nkv[t] = 0;
-    }
-  }
-  const int n_max = max(unit_nkv[0], unit_nkv[1]);
+  const int u0 = cta * NQ, u1 = cta * NQ + 1;
+  const int pb0 = u0 / p.group, pb1 = u1 / p.group;
+  const int head0 = kvh * p.group + (u0 - pb0 * p.group);
+  const int head1 = kvh * p.group + (u1 - pb1 * p.group);
+  auto n_tiles = [&](int pb) {
+    return p.causal ? min(p.n_kb, ((pb + 1) * BM + BN - 1) / BN) : p.n_kb;
+  };
+  const int nkv0 = (u0 < n_units) ? n_tiles(pb0) : 0;
+  const int nkv1 = (u1 < n_units) ? n_tiles(pb1) : 0;
+  const int n_max = max(nkv0, nkv1);
 
   // ---- setup
   if (threadIdx.x == 0) {
@@ -139,102 +143,134 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = s.tmem_base;
-  const uint32_t tm_s[NQ] = {tmem, tmem + BN};
-  const uint32_t tm_o[NQ] = {tmem + 2 * BN, tmem + 2 * BN + D};
+  // TMEM columns: S_0 [0,128), S_1 [128,256), O_0 [256,256+D), O_1 [256+D,256+2D)
+  auto tm_s = [&](int t) { return tmem + static_cast<uint32_t>(t * BN); };
+  auto tm_o = [&](int t) { return tmem + static_cast<uint32_t>(2 * BN + t * D); };
   if (warp == 0) {
     // ================================================================ TMA producer
+    // The whole warp runs the loop (waits and addresses stay warp-uniform);
+    // one elected lane issues the copies.
     setmaxnreg_dec<kRegsControl>();
-    if (lane == 0) {
+    if (elect_one()) {
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
-      int k_issued = 0, v_issued = 0;
-      for (int j = 0; j < n_max; ++j) {
-        const int ks = j % KSTAGES;
-        if (j >= KSTAGES && !mbar_wait(&s.k_empty[ks], ((j / KSTAGES) - 1) & 1)) break;
+    }
+    __syncwarp();
+    int k_issued = 0, v_issued = 0;
+    for (int j = 0; j < n_max; ++j) {
+      const int ks = j % KSTAGES;
+      if (j >= KSTAGES && !mbar_wait(&s.k_empty[ks], ((j / KSTAGES) - 1) & 1)) break;
+      if (elect_one()) {
         mbar_arrive_expect_tx(&s.k_full[ks], TILE_BYTES);
 #pragma unroll
         for (int cb = 0; cb < CB; ++cb)
           tma_load_4d(reinterpret_cast<uint8_t*>(&s.k[ks][0]) + cb * BLOCK_BYTES, &tm_k,
                       &s.k_full[ks], cb * 64, kvh, j * BN, b);
-        k_issued = j + 1;
-        const int vs = j % VSTAGES;
-        if (j >= VSTAGES && !mbar_wait(&s.v_empty[vs], ((j / VSTAGES) - 1) & 1)) break;
+      }
+      __syncwarp();
+      k_issued = j + 1;
+      const int vs = j % VSTAGES;
+      if (j >= VSTAGES && !mbar_wait(&s.v_empty[vs], ((j / VSTAGES) - 1) & 1)) break;
+      if (elect_one()) {
         mbar_arrive_expect_tx(&s.v_full[vs], TILE_BYTES);
 #pragma unroll
         for (int cb = 0; cb < CB; ++cb)
           tma_load_4d(reinterpret_cast<uint8_t*>(&s.v[vs][0]) + cb * BLOCK_BYTES, &tm_v,
                       &s.v_full[vs], cb * 64, kvh, j * BN, b);
-        v_issued = j + 1;
       }
-      // leave no copy in flight
-      for (int j = max(0, k_issued - KSTAGES); j < k_issued; ++j)
-        if (!mbar_wait(&s.k_full[j % KSTAGES], (j / KSTAGES) & 1)) break;
-      for (int j = max(0, v_issued - VSTAGES); j < v_issued; ++j)
-        if (!mbar_wait(&s.v_full[j % VSTAGES], (j / VSTAGES) & 1)) break;
+      __syncwarp();
+      v_issued = j + 1;
     }
+    // leave no copy in flight
+    for (int j = max(0, k_issued - KSTAGES); j < k_issued; ++j)
+      if (!mbar_wait(&s.k_full[j % KSTAGES], (j / KSTAGES) & 1)) break;
+    for (int j = max(0, v_issued - VSTAGES); j < v_issued; ++j)
+      if (!mbar_wait(&s.v_full[j % VSTAGES], (j / VSTAGES) & 1)) break;
   } else if (warp == 1) {
     // ================================================================ MMA issuer
+    // Converged warp, single elected issuing lane (tcgen05.mma and commit
+    // take warp-uniform operands).
     setmaxnreg_dec<kRegsControl>();
-    if (lane == 0) {
-      bool ok = true;
-      const uint32_t q_addr[NQ] = {smem_u32(&s.q[0][0]), smem_u32(&s.q[1][0])};
-      auto issue_qk = [&](int t, int ks) {
-        const uint32_t ka = smem_u32(&s.k[ks][0]);
+    bool ok = true;
+    const uint32_t q_base = smem_u32(&s.q[0][0]);
+    const uint32_t k_base = smem_u32(&s.k[0][0]);
+    const uint32_t v_base = smem_u32(&s.v[0][0]);
+    // descriptors of stage / tile bases; a k-step adds its byte offset >> 4 to
+    // the start-address field (the offsets stay inside one 16 KB block)
+    const uint64_t q_desc0 = sw128_desc(q_base, 16, 1024);
+    const uint64_t k_desc0 = sw128_desc(k_base, 16, 1024);
+    const uint64_t v_desc0 = sw128_desc(v_base, BLOCK_BYTES, 1024);
+    auto issue_qk = [&](int t, int ks) {
+      const uint64_t qd = q_desc0 + ((static_cast<uint32_t>(t) * TILE_BYTES) >> 4);
+      const uint64_t kd = k_desc0 + ((static_cast<uint32_t>(ks) * TILE_BYTES) >> 4);
+      if (elect_one()) {
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk / 4) * BLOCK_BYTES + (kk % 4) * 32;
-          mma_ss(tm_s[t], sw128_desc(q_addr[t] + off, 16, 1024), sw128_desc(ka + off, 16, 1024),
-                 IDESC_QK, kk > 0 ? 1u : 0u);
+          const uint32_t off = ((kk / 4) * BLOCK_BYTES + (kk % 4) * 32) >> 4;
+          mma_ss(tm_s(t), qd + off, kd + off, IDESC_QK, kk > 0 ? 1u : 0u);
         }
-      };
-      auto issue_pv = [&](int t, int vs, bool accumulate) {
-        const uint32_t va = smem_u32(&s.v[vs][0]);
+      }
+      __syncwarp();
+    };
+    auto issue_pv = [&](int t, int vs, bool accumulate) {
+      const uint64_t vd = v_desc0 + ((static_cast<uint32_t>(vs) * TILE_BYTES) >> 4);
+      if (elect_one()) {
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk) {
           // A = P_t[:, 16kk:16kk+16] in TMEM (8 columns of packed bf16 pairs);
           // B = V rows 16kk.. (MN-major: 64-dim blocks BLOCK_BYTES apart, 8-row groups 1 KB apart)
-          mma_ts(tm_o[t], tm_s[t] + kk * 8, sw128_desc(va + kk * 2048, BLOCK_BYTES, 1024),
-                 IDESC_PV, (accumulate || kk > 0) ? 1u : 0u);
+          mma_ts(tm_o(t), tm_s(t) + kk * 8, vd + ((kk * 2048) >> 4), IDESC_PV,
+                 (accumulate || kk > 0) ? 1u : 0u);
         }
-      };
-      for (int t = 0; t < NQ && ok; ++t)
-        if (unit_nkv[t] > 0) ok = mbar_wait(&s.q_ready[t], 0);
-      if (ok && n_max > 0) ok = mbar_wait(&s.k_full[0], 0);
-      if (ok && n_max > 0) {
-        tc_fence_after();
-        for (int t = 0; t < NQ; ++t)
-          if (unit_nkv[t] > 0) {
-            issue_qk(t, 0);
-            tc_commit(&s.s_full[t]);
-          }
-        tc_commit(&s.k_empty[0]);
       }
-      for (int j = 0; j < n_max && ok; ++j) {
-        const int vs = j % VSTAGES;
-        if (!mbar_wait(&s.v_full[vs], (j / VSTAGES) & 1)) { ok = false; break; }
-        const int jn = j + 1;
-        const bool next = jn < n_max;
-        if (next && !mbar_wait(&s.k_full[jn % KSTAGES], (jn / KSTAGES) & 1)) { ok = false; break; }
-        for (int t = 0; t < NQ; ++t) {
-          if (j >= unit_nkv[t]) continue;
-          if (!mbar_wait(&s.p_full[t], j & 1)) { ok = false; break; }
-          tc_fence_after();
-          issue_pv(t, vs, j > 0);
-          if (jn == unit_nkv[t]) {
-            tc_commit(&s.o_full[t]);
-          } else {
-            issue_qk(t, jn % KSTAGES);
-            tc_commit(&s.s_full[t]);
-          }
-        }
-        if (!ok) break;
-        tc_commit(&s.v_empty[vs]);
-        if (next) tc_commit(&s.k_empty[jn % KSTAGES]);
+      __syncwarp();
+    };
+    auto commit = [&](uint64_t* bar) {
+      if (elect_one()) tc_commit(bar);
+      __syncwarp();
+    };
+    if (nkv0 > 0) ok = mbar_wait(&s.q_ready[0], 0);
+    if (ok && nkv1 > 0) ok = mbar_wait(&s.q_ready[1], 0);
+    if (ok) ok = mbar_wait(&s.k_full[0], 0);
+    if (ok) {
+      tc_fence_after();
+      issue_qk(0, 0);
+      commit(&s.s_full[0]);
+      if (nkv1 > 0) {
+        issue_qk(1, 0);
+        commit(&s.s_full[1]);
       }
-      // every MMA this thread issued has completed before the CTA can exit
-      tc_commit(&s.mma_done);
-      mbar_wait(&s.mma_done, 0);
+      commit(&s.k_empty[0]);
     }
+    // one unit's step of iteration j: O_t += P_t V_j, then S_t = Q_t K_{j+1}^T
+    auto unit_step = [&](int t, int nkv, int j, int vs) -> bool {
+      if (j >= nkv) return true;
+      if (!mbar_wait(&s.p_full[t], j & 1)) return false;
+      tc_fence_after();
+      issue_pv(t, vs, j > 0);
+      if (j + 1 == nkv) {
+        commit(&s.o_full[t]);
+      } else {
+        issue_qk(t, (j + 1) % KSTAGES);
+        commit(&s.s_full[t]);
+      }
+      return true;
+    };
+    for (int j = 0; j < n_max && ok; ++j) {
+      const int vs = j % VSTAGES;
+      const int jn = j + 1;
+      const bool next = jn < n_max;
+      ok = mbar_wait(&s.v_full[vs], (j / VSTAGES) & 1);
+      if (ok && next) ok = mbar_wait(&s.k_full[jn % KSTAGES], (jn / KSTAGES) & 1);
+      if (ok) ok = unit_step(0, nkv0, j, vs);
+      if (ok) ok = unit_step(1, nkv1, j, vs);
+      if (!ok) break;
+      commit(&s.v_empty[vs]);
+      if (next) commit(&s.k_empty[jn % KSTAGES]);
+    }
+    // every MMA this warp issued has completed before the CTA can exit
+    commit(&s.mma_done);
+    mbar_wait(&s.mma_done, 0);
   } else if (warp < 4) {
     setmaxnreg_dec<kRegsControl>();  // idle warps of warpgroup 0
   } else {
@@ -243,10 +279,12 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
     const int t = (warp - 4) >> 2;     // unit handled by this warpgroup
     const int quarter = warp & 3;      // TMEM lane quarter of this warp
     const int r = quarter * 32 + lane; // row of the Q tile = TMEM lane
-    const int n_kv = unit_nkv[t];
+    const int n_kv = t ? nkv1 : nkv0;
+    const int my_pb = t ? pb1 : pb0;
+    const uint32_t my_s = tm_s(t), my_o = tm_o(t);
     if (n_kv > 0) {
-      const int head = unit_head[t];
-      const int i = unit_pb[t] * BM + r;  // query position (sequence index)
+      const int head = t ? head1 : head0;
+      const int i = my_pb * BM + r;  // query position (sequence index)
       const bool row_valid = i < p.S;
       // ---- stage Q: rotate this row and write it swizzled into s.q[t]
       {
@@ -299,74 +337,85 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
         tc_fence_after();
         uint32_t sr[4][32];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) tmem_ld32(tm_s[t] + lane_off + c * 32, sr[c]);
+        for (int c = 0; c < 4; ++c) tmem_ld32(my_s + lane_off + c * 32, sr[c]);
 #pragma unroll
         for (int c = 0; c < 4; ++c) tmem_ld_wait(sr[c]);
-        // v: raw scores (fast tiles: the scale is folded into the exponent's FMA) or
-        // scaled + masked scores (tiles that touch the diagonal, the ragged end or a mask)
-        float v[BN];
+        // v: raw scores (interior tiles: the scale is folded into the exponent's FMA)
+        // or scaled + masked scores (tiles that touch the diagonal, the ragged end
+        // or a mask, and any tile when scale <= 0)
         const int key0 = j * BN;
-        const bool edge = (key0 + BN > p.S) || (p.causal && key0 + BN - 1 > unit_pb[t] * BM) ||
+        const bool edge = (key0 + BN > p.S) || (p.causal && key0 + BN - 1 > my_pb * BM) ||
                           (mrow != nullptr) || !scale_pos;
-        if (!edge) {
-#pragma unroll
-          for (int e = 0; e < BN; ++e) v[e] = __uint_as_float(sr[e / 32][e % 32]);
-        } else {
-          const int lim = p.causal ? min(p.S - 1, i) : p.S - 1;  // last visible key
-#pragma unroll
-          for (int e = 0; e < BN; ++e) {
-            const int key = key0 + e;
-            float xv = __uint_as_float(sr[e / 32][e % 32]) * c_log2;
-            if (mrow != nullptr && key < p.S) xv = fmaf(mrow[key], 1.4426950408889634f, xv);
-            v[e] = (key <= lim) ? xv : -INFINITY;
-          }
-        }
-        // row max: eight independent 3-input chains, then a small tree
-        float mm[8];
-#pragma unroll
-        for (int k = 0; k < 8; ++k) mm[k] = fmaxf(v[k], v[k + 8]);
-#pragma unroll
-        for (int e = 16; e < BN; e += 16)
-#pragma unroll
-          for (int k = 0; k < 8; ++k) mm[k] = fmax3f(mm[k], v[e + k], v[e + k + 8]);
-        float mx = fmax3f(fmax3f(mm[0], mm[1], mm[2]), fmax3f(mm[3], mm[4], mm[5]), fmaxf(mm[6], mm[7]));
-        if (!edge) mx *= c_log2;
-        // lazy reference: move only when the max grows by more than the threshold
-        float alpha = 1.f;
-        if (mx > m_ref + kRescaleThreshold || (m_ref == -INFINITY && mx != -INFINITY)) {
-          alpha = (m_ref == -INFINITY) ? 0.f : ex2_approx(m_ref - mx);
-          m_ref = mx;
-        }
-        const float nref = (m_ref == -INFINITY) ? 0.f : -m_ref;
-        const float cc = edge ? 1.f : c_log2;
+        float alpha = 1.f, rs = 0.f;
         uint32_t pk[2][32];
-        float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        auto tile = [&](auto edge_c) {
+          constexpr bool kEdge = decltype(edge_c)::value;
+          float v[BN];
+          if (!kEdge) {
 #pragma unroll
-        for (int e = 0; e < BN; e += 2) {
-          float a0, a1;
-          ffma2(a0, a1, v[e], v[e + 1], cc, cc, nref, nref);  // exponent = v*c - m_ref
-          const float p0 = ex2_approx(a0);
-          const float p1 = ex2_approx(a1);
-          const int k = (e / 2) % 4;
-          fadd2(acc[2 * k], acc[2 * k + 1], acc[2 * k], acc[2 * k + 1], p0, p1);
-          pk[e / 64][(e % 64) / 2] = pack_bf16x2(p0, p1);
-        }
-        const float rs = ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
+            for (int e = 0; e < BN; ++e) v[e] = __uint_as_float(sr[e / 32][e % 32]);
+          } else {
+            const int lim = p.causal ? min(p.S - 1, i) : p.S - 1;  // last visible key
+#pragma unroll
+            for (int e = 0; e < BN; ++e) {
+              const int key = key0 + e;
+              float xv = __uint_as_float(sr[e / 32][e % 32]) * c_log2;
+              if (mrow != nullptr && key < p.S) xv = fmaf(mrow[key], 1.4426950408889634f, xv);
+              v[e] = (key <= lim) ? xv : -INFINITY;
+            }
+          }
+          // row max: eight independent 3-input chains, then a small tree
+          float mm[8];
+#pragma unroll
+          for (int k = 0; k < 8; ++k) mm[k] = fmaxf(v[k], v[k + 8]);
+#pragma unroll
+          for (int e = 16; e < BN; e += 16)
+#pragma unroll
+            for (int k = 0; k < 8; ++k) mm[k] = fmax3f(mm[k], v[e + k], v[e + k + 8]);
+          float mx = fmax3f(fmax3f(mm[0], mm[1], mm[2]), fmax3f(mm[3], mm[4], mm[5]),
+                            fmaxf(mm[6], mm[7]));
+          if (!kEdge) mx *= c_log2;
+          // lazy reference: move only when the max grows by more than the threshold
+          if (mx > m_ref + kRescaleThreshold || (m_ref == -INFINITY && mx != -INFINITY)) {
+            alpha = (m_ref == -INFINITY) ? 0.f : ex2_approx(m_ref - mx);
+            m_ref = mx;
+          }
+          const float nref = (m_ref == -INFINITY) ? 0.f : -m_ref;
+          const float cc = kEdge ? 1.f : c_log2;
+          float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+          for (int e = 0; e < BN; e += 2) {
+            float a0, a1, p0, p1;
+            ffma2(a0, a1, v[e], v[e + 1], cc, cc, nref, nref);  // exponent = v*c - m_ref
+            if (!kEdge && ((e / 2) % 8) < kPolyPairsOf8) {
+              exp2_poly2(p0, p1, a0, a1);
+            } else {
+              p0 = ex2_approx(a0);
+              p1 = ex2_approx(a1);
+            }
+            const int k = (e / 2) % 4;
+            fadd2(acc[2 * k], acc[2 * k + 1], acc[2 * k], acc[2 * k + 1], p0, p1);
+            pk[e / 64][(e % 64) / 2] = pack_bf16x2(p0, p1);
+          }
+          rs = ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
+        };
+        if (edge) tile(std::true_type{});
+        else tile(std::false_type{});
         l_sum = fmaf(l_sum, alpha, rs);
         // O correction (warp-collective TMEM access when any row of the warp needs it)
         if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll
           for (int c = 0; c < D / 32; ++c) {
             uint32_t orr[32];
-            tmem_ld32(tm_o[t] + lane_off + c * 32, orr);
+            tmem_ld32(my_o + lane_off + c * 32, orr);
             tmem_ld_wait(orr);
 #pragma unroll
             for (int e = 0; e < 32; ++e) orr[e] = __float_as_uint(__uint_as_float(orr[e]) * alpha);
-            tmem_st32(tm_o[t] + lane_off + c * 32, orr);
+            tmem_st32(my_o + lane_off + c * 32, orr);
           }
         }
-        tmem_st32(tm_s[t] + lane_off, pk[0]);
-        tmem_st32(tm_s[t] + lane_off + 32, pk[1]);
+        tmem_st32(my_s + lane_off, pk[0]);
+        tmem_st32(my_s + lane_off + 32, pk[1]);
         tmem_st_wait();
         tc_fence_before();
         mbar_arrive(&s.p_full[t]);
@@ -380,7 +429,7 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
           uint32_t orr[32];
-          tmem_ld32(tm_o[t] + lane_off + c * 32, orr);
+          tmem_ld32(my_o + lane_off + c * 32, orr);
           tmem_ld_wait(orr);
           if (row_valid) {
 #pragma unroll
