@@ -80,14 +80,15 @@ struct PfSmem {
   alignas(1024) __nv_bfloat16 v[pf::VSTAGES][pf::BN * D];
   uint64_t k_full[pf::KSTAGES], k_empty[pf::KSTAGES];
   uint64_t v_full[pf::VSTAGES], v_empty[pf::VSTAGES];
-  uint64_t q_ready[pf::NQ], s_full[pf::NQ], p_full[pf::NQ], o_full[pf::NQ];
+  uint64_t q_loaded[pf::NQ], q_ready[pf::NQ], s_full[pf::NQ], p_full[pf::NQ], o_full[pf::NQ];
   uint64_t mma_done;
   uint32_t tmem_base;
 };
 
 template <int D>
 __global__ void __launch_bounds__(pf::THREADS, 1)
-    prefill_sm100_kernel(const __grid_constant__ CUtensorMap tm_k,
+    prefill_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
+                         const __grid_constant__ CUtensorMap tm_k,
                          const __grid_constant__ CUtensorMap tm_v, PrefillParams p) {
   using namespace pf;
   constexpr int CB = D / 64;                       // 64-column swizzle blocks per row
@@ -127,7 +128,8 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
     for (int i = 0; i < KSTAGES; ++i) { mbar_init(&s.k_full[i], 1); mbar_init(&s.k_empty[i], 1); }
     for (int i = 0; i < VSTAGES; ++i) { mbar_init(&s.v_full[i], 1); mbar_init(&s.v_empty[i], 1); }
     for (int t = 0; t < NQ; ++t) {
-      mbar_init(&s.q_ready[t], 128);
+      mbar_init(&s.q_loaded[t], 1);
+      mbar_init(&s.q_ready[t], 4);
       mbar_init(&s.s_full[t], 1);
       mbar_init(&s.p_full[t], 128);
       mbar_init(&s.o_full[t], 1);
@@ -152,8 +154,22 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
     // one elected lane issues the copies.
     setmaxnreg_dec<kRegsControl>();
     if (elect_one()) {
+      tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
+      // the two Q tiles (raw; rotated in shared memory by their softmax warps)
+      mbar_arrive_expect_tx(&s.q_loaded[0], TILE_BYTES);
+#pragma unroll
+      for (int cb = 0; cb < CB; ++cb)
+        tma_load_4d(reinterpret_cast<uint8_t*>(&s.q[0][0]) + cb * BLOCK_BYTES, &tm_q,
+                    &s.q_loaded[0], cb * 64, head0, pb0 * BM, b);
+      if (nkv1 > 0) {
+        mbar_arrive_expect_tx(&s.q_loaded[1], TILE_BYTES);
+#pragma unroll
+        for (int cb = 0; cb < CB; ++cb)
+          tma_load_4d(reinterpret_cast<uint8_t*>(&s.q[1][0]) + cb * BLOCK_BYTES, &tm_q,
+                      &s.q_loaded[1], cb * 64, head1, pb1 * BM, b);
+      }
     }
     __syncwarp();
     int k_issued = 0, v_issued = 0;
@@ -182,6 +198,8 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
       v_issued = j + 1;
     }
     // leave no copy in flight
+    mbar_wait(&s.q_loaded[0], 0);
+    if (nkv1 > 0) mbar_wait(&s.q_loaded[1], 0);
     for (int j = max(0, k_issued - KSTAGES); j < k_issued; ++j)
       if (!mbar_wait(&s.k_full[j % KSTAGES], (j / KSTAGES) & 1)) break;
     for (int j = max(0, v_issued - VSTAGES); j < v_issued; ++j)
@@ -286,43 +304,47 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
       const int head = t ? head1 : head0;
       const int i = my_pb * BM + r;  // query position (sequence index)
       const bool row_valid = i < p.S;
-      // ---- stage Q: rotate this row and write it swizzled into s.q[t]
+      // ---- stage Q: the raw tile arrives by TMA; rotate it in shared memory.
+      // Warp-cooperative: per step a warp takes 32 / (D/4) rows, each lane one
+      // bf16 pair (d, d+1) of the first half and its partner pair d + D/2, with
+      // coalesced cos/sin loads; 32 lanes cover whole 128-byte rows, so the
+      // swizzled accesses are free of bank conflicts.
       {
-        uint8_t* qs = reinterpret_cast<uint8_t*>(&s.q[t][0]);
-        const __nv_bfloat16* qr = p.q + ((static_cast<size_t>(b) * p.S + i) * p.H + head) * D;
-        const float* cr = p.cos ? p.cos + (static_cast<size_t>(b) * p.S + i) * D : nullptr;
-        const float* sr = p.sin ? p.sin + (static_cast<size_t>(b) * p.S + i) * D : nullptr;
-#pragma unroll
-        for (int c = 0; c < D / 16; ++c) {  // chunk c of the first half, c + D/16 of the second
-          uint4 lo = make_uint4(0, 0, 0, 0), hi = make_uint4(0, 0, 0, 0);
-          if (row_valid) {
-            const uint4 a = *reinterpret_cast<const uint4*>(qr + c * 8);
-            const uint4 z = *reinterpret_cast<const uint4*>(qr + D / 2 + c * 8);
-            if (cr) {
-              const uint32_t au[4] = {a.x, a.y, a.z, a.w}, zu[4] = {z.x, z.y, z.z, z.w};
-              uint32_t lu[4], hu[4];
-#pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                const int d = c * 8 + 2 * e;
-                const float x0 = bf16lo(au[e]), x1 = bf16hi(au[e]);
-                const float z0 = bf16lo(zu[e]), z1 = bf16hi(zu[e]);
-                lu[e] = pack_bf16x2(fmaf(x0, cr[d], -z0 * sr[d]), fmaf(x1, cr[d + 1], -z1 * sr[d + 1]));
-                hu[e] = pack_bf16x2(fmaf(z0, cr[d + D / 2], x0 * sr[d + D / 2]),
-                                    fmaf(z1, cr[d + D / 2 + 1], x1 * sr[d + D / 2 + 1]));
-              }
-              lo = make_uint4(lu[0], lu[1], lu[2], lu[3]);
-              hi = make_uint4(hu[0], hu[1], hu[2], hu[3]);
-            } else {
-              lo = a;
-              hi = z;
-            }
+        if (!mbar_wait(&s.q_loaded[t], 0)) {
+          // fall through: the loop below will see its own waits time out
+        } else if (p.cos != nullptr) {
+          constexpr int PAIRS = D / 4;             // bf16 pairs in half a row
+          constexpr int ROWS_PER_STEP = 32 / PAIRS;
+          uint8_t* qs = reinterpret_cast<uint8_t*>(&s.q[t][0]);
+          const int wq = warp & 3;                 // warp index inside the warpgroup
+          const int pr = lane % PAIRS, rsub = lane / PAIRS;
+          const int d = 2 * pr;                    // first-half dim of this lane's pair
+          const int d2 = d + D / 2;                // its rotation partner
+          const uint32_t colb = static_cast<uint32_t>((d % 64) / 8), inb = (d % 8) * 2;
+          const uint32_t colb2 = static_cast<uint32_t>((d2 % 64) / 8);
+#pragma unroll 4
+          for (int rr = wq * 32 + rsub; rr < wq * 32 + 32; rr += ROWS_PER_STEP) {
+            const int pos = my_pb * BM + rr;
+            if (pos >= p.S) continue;
+            const size_t trow = (static_cast<size_t>(b) * p.S + pos) * D;
+            const float2 c1 = *reinterpret_cast<const float2*>(p.cos + trow + d);
+            const float2 c2 = *reinterpret_cast<const float2*>(p.cos + trow + d2);
+            const float2 s1 = *reinterpret_cast<const float2*>(p.sin + trow + d);
+            const float2 s2 = *reinterpret_cast<const float2*>(p.sin + trow + d2);
+            const uint32_t row = static_cast<uint32_t>(rr) * 128;
+            uint32_t* p1 = reinterpret_cast<uint32_t*>(qs + (d / 64) * BLOCK_BYTES + row +
+                                                       (((colb ^ (rr & 7)) << 4) | inb));
+            uint32_t* p2 = reinterpret_cast<uint32_t*>(qs + (d2 / 64) * BLOCK_BYTES + row +
+                                                       (((colb2 ^ (rr & 7)) << 4) | inb));
+            const uint32_t xa = *p1, za = *p2;
+            const float x0 = bf16lo(xa), x1 = bf16hi(xa), z0 = bf16lo(za), z1 = bf16hi(za);
+            *p1 = pack_bf16x2(fmaf(x0, c1.x, -z0 * s1.x), fmaf(x1, c1.y, -z1 * s1.y));
+            *p2 = pack_bf16x2(fmaf(z0, c2.x, x0 * s2.x), fmaf(z1, c2.y, x1 * s2.y));
           }
-          const int c2 = c + D / 16;
-          *reinterpret_cast<uint4*>(qs + (c / 8) * BLOCK_BYTES + sw128_offset(r, c % 8)) = lo;
-          *reinterpret_cast<uint4*>(qs + (c2 / 8) * BLOCK_BYTES + sw128_offset(r, c2 % 8)) = hi;
+          fence_proxy_async_smem();
         }
-        fence_proxy_async_smem();
-        mbar_arrive(&s.q_ready[t]);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&s.q_ready[t]);
       }
 
       const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
