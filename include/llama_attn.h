@@ -126,6 +126,33 @@ int llama_attn_decode(const void* q, const void* k_cache, const void* v_cache,
                       float scale, void* out, void* workspace, size_t workspace_bytes,
                       int dtype, void* cuda_stream);
 
+/*
+ * Single-token decode for callers that cannot allocate device memory.  The
+ * pages have no counterpart to this entry point; it exists for integrations
+ * that hand the library only their input and output buffers -- hosts that
+ * reserve all device memory up front and forbid further cudaMalloc (which
+ * could also synchronise the device mid-step), or plugin interfaces that
+ * provide no workspace.  It computes exactly what llama_attn_decode computes,
+ * with the same arguments minus the workspace.
+ *
+ * Scratch: a file-scope device array of 16 MiB inside the library, which every
+ * GPU that loads the library holds until the process exits.  A request needing
+ * more than that (see llama_attn_decode_workspace_bytes) is rejected with
+ * LLAMA_ERR_INVALID_ARG before anything is enqueued; use llama_attn_decode
+ * with a caller workspace instead.  fp32 requests need no scratch.
+ * The first call on a device looks up the array's device address (one
+ * cudaGetSymbolAddress, no allocation); make that first call before any
+ * stream capture on that device.
+ * Every call on a device shares the one array and leaves its last contents
+ * behind (each call writes every scratch entry it later reads, so nothing has
+ * to start at zero).  Calls whose kernels overlap on the GPU -- concurrent
+ * streams, or several host threads -- race on the array: serialise them.
+ */
+int llama_attn_decode_noalloc(const void* q, const void* k_cache, const void* v_cache,
+                              const int* cache_lens, const float* cos, const float* sin, int bsz,
+                              int n_heads, int n_kv_heads, int max_cache_len, int head_dim,
+                              float scale, void* out, int dtype, void* cuda_stream);
+
 /* Synchronises `cuda_stream`, then reads and clears the device status word of
  * the current device.  Returns LLAMA_OK, LLAMA_ERR_DEVICE_TIMEOUT, or
  * LLAMA_ERR_CUDA if the synchronisation itself failed. */

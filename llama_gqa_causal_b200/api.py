@@ -34,6 +34,7 @@ EXPORTED = (
     "llama_attn_prefill",
     "llama_attn_decode_workspace_bytes",
     "llama_attn_decode",
+    "llama_attn_decode_noalloc",
     "llama_attn_device_status",
     "llama_attn_status_string",
     "llama_attn_abi_version",
@@ -68,6 +69,8 @@ def load() -> ctypes.CDLL:
     lib.llama_attn_decode_workspace_bytes.restype = Z
     lib.llama_attn_decode.argtypes = [P, P, P, P, P, P, I, I, I, I, I, F, P, P, Z, I, P]
     lib.llama_attn_decode.restype = I
+    lib.llama_attn_decode_noalloc.argtypes = [P, P, P, P, P, P, I, I, I, I, I, F, P, I, P]
+    lib.llama_attn_decode_noalloc.restype = I
     lib.llama_attn_device_status.argtypes = [P]
     lib.llama_attn_device_status.restype = I
     lib.llama_attn_status_string.argtypes = [I]
@@ -181,6 +184,29 @@ def decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
                                  _ptr(cos), _ptr(sin), b, H, Hkv, L, D, float(scale), _ptr(out),
                                  _ptr(workspace), ws_bytes, _dtype_code(q.dtype),
                                  _stream(stream)), "llama_attn_decode")
+    return out
+
+
+def decode_noalloc(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+                   cache_lens: torch.Tensor, cos: Optional[torch.Tensor] = None,
+                   sin: Optional[torch.Tensor] = None, *, scale: Optional[float] = None,
+                   out: torch.Tensor, stream=None) -> torch.Tensor:
+    """llama_attn_decode_noalloc: decode with the library's static scratch.
+
+    For callers that must not allocate device memory: ``out`` is required
+    (shape [b, H*D], same dtype as q) and nothing is allocated here either.
+    """
+    lib = load()
+    b, H, D = q.shape
+    Hkv, L = k_cache.shape[1], k_cache.shape[2]
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    if cache_lens.dtype != torch.int32:
+        raise ValueError("llama_attn_decode_noalloc: cache_lens must be int32")
+    _check(lib.llama_attn_decode_noalloc(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(cache_lens),
+                                         _ptr(cos), _ptr(sin), b, H, Hkv, L, D, float(scale),
+                                         _ptr(out), _dtype_code(q.dtype), _stream(stream)),
+           "llama_attn_decode_noalloc")
     return out
 
 

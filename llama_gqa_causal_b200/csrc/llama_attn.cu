@@ -212,6 +212,36 @@ int decode_bf16(const void* q, const void* kc, const void* vc, const int* lens, 
 
 }  // namespace
 
+// ---------------------------------------------------------------- decode without caller scratch
+// Split-KV decode needs a scratch area for its per-split partial results.
+// llama_attn_decode_noalloc takes it from this array instead of from the
+// caller: it lives in the library's device image, so every GPU that loads the
+// library holds it until the process exits.
+namespace {
+constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;  // 16 MiB per GPU
+}
+static __device__ __align__(256) unsigned char g_decode_noalloc_scratch[kNoAllocScratchBytes];
+
+namespace {
+// Device address of the scratch array on the current device.  Host code may
+// not use the array's name as a pointer (on the host it is only a stand-in
+// for the symbol), so the address is looked up once per device, with that
+// device current, and cached.
+void* noalloc_scratch_for_current_device() {
+  static std::mutex mu;
+  static void* addr[64] = {};
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if (addr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_decode_noalloc_scratch) != cudaSuccess) return nullptr;
+    addr[dev] = p;
+  }
+  return addr[dev];
+}
+}  // namespace
+
 extern "C" {
 
 int llama_attn_abi_version(void) { return kAbiVersion; }
@@ -319,6 +349,33 @@ int llama_attn_decode(const void* q, const void* k_cache, const void* v_cache,
   return attn_fp32<64>(qf, static_cast<const float*>(k_cache), static_cast<const float*>(v_cache),
                        cos, sin, nullptr, cache_lens, static_cast<float*>(out), bsz, n_heads,
                        n_kv_heads, 1, max_cache_len, 1, 0, scale, st);
+}
+
+int llama_attn_decode_noalloc(const void* q, const void* k_cache, const void* v_cache,
+                              const int* cache_lens, const float* cos, const float* sin, int bsz,
+                              int n_heads, int n_kv_heads, int max_cache_len, int head_dim,
+                              float scale, void* out, int dtype, void* cuda_stream) {
+  if (dtype == LLAMA_DT_BF16) {
+    // reject requests the static scratch cannot hold before touching the device
+    if (bsz >= 1 && n_heads >= 1 && max_cache_len >= 1 && head_dim >= 1 &&
+        llama_attn_decode_workspace_bytes(bsz, n_heads, max_cache_len, head_dim) >
+            kNoAllocScratchBytes) {
+      fprintf(stderr,
+              "llama_attn_decode_noalloc: %zu bytes of scratch needed, the static limit is %zu; "
+              "use llama_attn_decode with a caller workspace\n",
+              llama_attn_decode_workspace_bytes(bsz, n_heads, max_cache_len, head_dim),
+              kNoAllocScratchBytes);
+      return LLAMA_ERR_INVALID_ARG;
+    }
+  }
+  void* scratch = nullptr;
+  if (dtype == LLAMA_DT_BF16 && q && k_cache && v_cache && cache_lens && out) {
+    scratch = noalloc_scratch_for_current_device();
+    if (scratch == nullptr) return LLAMA_ERR_CUDA;
+  }
+  return llama_attn_decode(q, k_cache, v_cache, cache_lens, cos, sin, bsz, n_heads, n_kv_heads,
+                           max_cache_len, head_dim, scale, out, scratch,
+                           scratch ? kNoAllocScratchBytes : 0, dtype, cuda_stream);
 }
 
 int llama_attn_device_status(void* cuda_stream) {

@@ -133,6 +133,15 @@ def test_rope_table_rejects(lib, args):
     assert lib.llama_rope_table(*args, None) == 1
 
 
+def test_decode_noalloc_refuses_what_its_static_scratch_cannot_hold(lib):
+    # 272 MB of split partials needed; the library's fixed scratch is 16 MiB
+    assert lib.llama_attn_decode_noalloc(FAKE, FAKE, FAKE, FAKE, None, None, 64, 64, 8, 65536, 128,
+                                         0.088, FAKE, 1, None) == 1
+    # argument checks are the regular decode's
+    assert lib.llama_attn_decode_noalloc(FAKE, FAKE, FAKE, None, None, None, 2, 8, 2, 100, 128,
+                                         0.1, FAKE, 1, None) == 1
+
+
 def test_python_binding_refuses_cpu_tensors(lib):
     import torch
     q = torch.zeros(1, 4, 2, 64, dtype=torch.bfloat16)
