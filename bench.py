@@ -45,6 +45,24 @@ DECODE = W.DECODE70B
 METRIC = "causal GQA prefill TFLOP/s and KV-decode HBM GB/s, % of B200 roofline"
 
 
+def _traffic(kernel: str):
+    """Per-launch DRAM bytes of `kernel` from the committed ncu record, or None
+    when the CUDA sources changed since that capture."""
+    import glob
+    import hashlib
+    try:
+        rec = json.load(open(os.path.join(ROOT, "profiles", "ncu_traffic.json")))
+    except Exception:
+        return None
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "llama_gqa_causal_b200", "csrc")
+    for f in sorted(glob.glob(os.path.join(csrc, "*.cu")) + glob.glob(os.path.join(csrc, "*.cuh"))):
+        h.update(open(f, "rb").read())
+    if h.hexdigest()[:16] != rec.get("csrc_sha256_16") or kernel not in rec:
+        return None
+    return rec[kernel]["dram_read_bytes"] + rec[kernel]["dram_write_bytes"]
+
+
 def _peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -262,7 +280,8 @@ def _prefill_phase(args, ws, local, dev, stream, line):
             "unit": "TFLOP/s",
             "frac": round(achieved / peak_burst, 4),
             "peak_source": f"{peak_src} bf16 burst",
-            "traffic": None,
+            "traffic": _traffic("prefill_sm100_kernel<128>"),
+            "traffic_unit": "bytes per launch (ncu dram read+write)",
         },
         "e2e": {
             "value": None if e2e_value is None else round(e2e_value, 3),
@@ -369,7 +388,7 @@ def _oracle_sample_prefill(cfg, rows):
 def cpu_baseline(rows=None):
     import oracle
     cfg = PREFILL
-    rows = rows or (cfg.seq - 16, cfg.seq)
+    rows = rows or (cfg.seq - 1024, cfg.seq)
     dt, flops = _oracle_sample_prefill(cfg, rows)
     return {"value": round(flops / dt / 1e12, 6), "unit": "TFLOP/s", "cores": oracle.max_threads(),
             "kind": "oracle",
