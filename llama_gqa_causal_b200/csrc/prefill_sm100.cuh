@@ -43,8 +43,14 @@ namespace pf {
 constexpr int BM = 128;       // query rows per tile (= TMEM lanes)
 constexpr int BN = 128;       // keys per K/V tile
 constexpr int NQ = 2;         // Q tiles (units) per CTA
-constexpr int KSTAGES = 2;
-constexpr int VSTAGES = 2;
+#ifndef LA_PF_KSTAGES
+#define LA_PF_KSTAGES 2
+#endif
+#ifndef LA_PF_VSTAGES
+#define LA_PF_VSTAGES 2
+#endif
+constexpr int KSTAGES = LA_PF_KSTAGES;  // K tile ring depth
+constexpr int VSTAGES = LA_PF_VSTAGES;  // V tile ring depth
 constexpr int THREADS = 384;  // warpgroup 0: TMA + MMA warps; warpgroups 1, 2: softmax
 // Register budget per warpgroup after setmaxnreg: each SMSP holds one warp of
 // every warpgroup, 56 + 224 + 224 registers x 32 lanes = 16128 <= 16384.
@@ -54,7 +60,7 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 units
 // Of every 8 consecutive pairs of probabilities in an interior tile, this
 // many are exponentiated on the FMA pipe (exp2_poly2), the rest on MUFU.
 #ifndef LA_POLY_PAIRS_OF_8
-#define LA_POLY_PAIRS_OF_8 2
+#define LA_POLY_PAIRS_OF_8 3
 #endif
 constexpr int kPolyPairsOf8 = LA_POLY_PAIRS_OF_8;
 }  // namespace pf
@@ -80,7 +86,8 @@ struct PfSmem {
   alignas(1024) __nv_bfloat16 v[pf::VSTAGES][pf::BN * D];
   uint64_t k_full[pf::KSTAGES], k_empty[pf::KSTAGES];
   uint64_t v_full[pf::VSTAGES], v_empty[pf::VSTAGES];
-  uint64_t q_loaded[pf::NQ], q_ready[pf::NQ], s_full[pf::NQ], p_full[pf::NQ], o_full[pf::NQ];
+  uint64_t q_loaded[pf::NQ], q_ready[pf::NQ], s_full[pf::NQ], p_lo[pf::NQ], p_hi[pf::NQ];
+  uint64_t o_full[pf::NQ];
   uint64_t mma_done;
   uint32_t tmem_base;
 };
@@ -131,7 +138,8 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
       mbar_init(&s.q_loaded[t], 1);
       mbar_init(&s.q_ready[t], 4);
       mbar_init(&s.s_full[t], 1);
-      mbar_init(&s.p_full[t], 128);
+      mbar_init(&s.p_lo[t], 4);
+      mbar_init(&s.p_hi[t], 4);
       mbar_init(&s.o_full[t], 1);
     }
     mbar_init(&s.mma_done, 1);
@@ -230,15 +238,16 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
       }
       __syncwarp();
     };
-    auto issue_pv = [&](int t, int vs, bool accumulate) {
+    // half h of O_t += P_t V: keys [64h, 64h + 64)
+    auto issue_pv = [&](int t, int vs, bool accumulate, int h) {
       const uint64_t vd = v_desc0 + ((static_cast<uint32_t>(vs) * TILE_BYTES) >> 4);
       if (elect_one()) {
 #pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk) {
+        for (int kk = h * (BN / 32); kk < (h + 1) * (BN / 32); ++kk) {
           // A = P_t[:, 16kk:16kk+16] in TMEM (8 columns of packed bf16 pairs);
           // B = V rows 16kk.. (MN-major: 64-dim blocks BLOCK_BYTES apart, 8-row groups 1 KB apart)
           mma_ts(tm_o(t), tm_s(t) + kk * 8, vd + ((kk * 2048) >> 4), IDESC_PV,
-                 (accumulate || kk > 0) ? 1u : 0u);
+                 (accumulate || kk > h * (BN / 32)) ? 1u : 0u);
         }
       }
       __syncwarp();
@@ -260,15 +269,33 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
       }
       commit(&s.k_empty[0]);
     }
-    // one unit's step of iteration j: O_t += P_t V_j, then S_t = Q_t K_{j+1}^T
+    // one unit's step of iteration j: O_t += P_t V_j, then S_t = Q_t K_{j+1}^T.
+    // V_j and K_{j+1} are waited for only right before their first use.
+    bool v_ready = false, k_ready = false;
+#ifdef LA_PF_MMA_SPIN
+    auto pwait = [&](uint64_t* bar, uint32_t par) { return mbar_wait_spin(bar, par); };
+#else
+    auto pwait = [&](uint64_t* bar, uint32_t par) { return mbar_wait(bar, par); };
+#endif
     auto unit_step = [&](int t, int nkv, int j, int vs) -> bool {
       if (j >= nkv) return true;
-      if (!mbar_wait(&s.p_full[t], j & 1)) return false;
+      if (!pwait(&s.p_lo[t], j & 1)) return false;
+      if (!v_ready) {
+        if (!mbar_wait(&s.v_full[vs], (j / VSTAGES) & 1)) return false;
+        v_ready = true;
+      }
       tc_fence_after();
-      issue_pv(t, vs, j > 0);
+      issue_pv(t, vs, j > 0, 0);
+      if (!pwait(&s.p_hi[t], j & 1)) return false;
+      tc_fence_after();
+      issue_pv(t, vs, true, 1);
       if (j + 1 == nkv) {
         commit(&s.o_full[t]);
       } else {
+        if (!k_ready) {
+          if (!mbar_wait(&s.k_full[(j + 1) % KSTAGES], ((j + 1) / KSTAGES) & 1)) return false;
+          k_ready = true;
+        }
         issue_qk(t, (j + 1) % KSTAGES);
         commit(&s.s_full[t]);
       }
@@ -278,9 +305,9 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
       const int vs = j % VSTAGES;
       const int jn = j + 1;
       const bool next = jn < n_max;
-      ok = mbar_wait(&s.v_full[vs], (j / VSTAGES) & 1);
-      if (ok && next) ok = mbar_wait(&s.k_full[jn % KSTAGES], (jn / KSTAGES) & 1);
-      if (ok) ok = unit_step(0, nkv0, j, vs);
+      v_ready = false;
+      k_ready = false;
+      ok = unit_step(0, nkv0, j, vs);
       if (ok) ok = unit_step(1, nkv1, j, vs);
       if (!ok) break;
       commit(&s.v_empty[vs]);
@@ -308,13 +335,16 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
       // Warp-cooperative: per step a warp takes 32 / (D/4) rows, each lane one
       // bf16 pair (d, d+1) of the first half and its partner pair d + D/2, with
       // coalesced cos/sin loads; 32 lanes cover whole 128-byte rows, so the
-      // swizzled accesses are free of bank conflicts.
+      // swizzled accesses are free of bank conflicts.  The cos/sin values of
+      // half the warp's rows are loaded into registers at once (the first half
+      // while the Q copy is still in flight), so the table reads cost two
+      // round trips rather than one per row.
       {
-        if (!mbar_wait(&s.q_loaded[t], 0)) {
-          // fall through: the loop below will see its own waits time out
-        } else if (p.cos != nullptr) {
+        if (p.cos != nullptr) {
           constexpr int PAIRS = D / 4;             // bf16 pairs in half a row
           constexpr int ROWS_PER_STEP = 32 / PAIRS;
+          constexpr int STEPS = 32 / ROWS_PER_STEP;  // steps covering the warp's 32 rows
+          constexpr int BATCH = STEPS / 2;
           uint8_t* qs = reinterpret_cast<uint8_t*>(&s.q[t][0]);
           const int wq = warp & 3;                 // warp index inside the warpgroup
           const int pr = lane % PAIRS, rsub = lane / PAIRS;
@@ -322,26 +352,40 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
           const int d2 = d + D / 2;                // its rotation partner
           const uint32_t colb = static_cast<uint32_t>((d % 64) / 8), inb = (d % 8) * 2;
           const uint32_t colb2 = static_cast<uint32_t>((d2 % 64) / 8);
-#pragma unroll 4
-          for (int rr = wq * 32 + rsub; rr < wq * 32 + 32; rr += ROWS_PER_STEP) {
-            const int pos = my_pb * BM + rr;
-            if (pos >= p.S) continue;
-            const size_t trow = (static_cast<size_t>(b) * p.S + pos) * D;
-            const float2 c1 = *reinterpret_cast<const float2*>(p.cos + trow + d);
-            const float2 c2 = *reinterpret_cast<const float2*>(p.cos + trow + d2);
-            const float2 s1 = *reinterpret_cast<const float2*>(p.sin + trow + d);
-            const float2 s2 = *reinterpret_cast<const float2*>(p.sin + trow + d2);
-            const uint32_t row = static_cast<uint32_t>(rr) * 128;
-            uint32_t* p1 = reinterpret_cast<uint32_t*>(qs + (d / 64) * BLOCK_BYTES + row +
-                                                       (((colb ^ (rr & 7)) << 4) | inb));
-            uint32_t* p2 = reinterpret_cast<uint32_t*>(qs + (d2 / 64) * BLOCK_BYTES + row +
-                                                       (((colb2 ^ (rr & 7)) << 4) | inb));
-            const uint32_t xa = *p1, za = *p2;
-            const float x0 = bf16lo(xa), x1 = bf16hi(xa), z0 = bf16lo(za), z1 = bf16hi(za);
-            *p1 = pack_bf16x2(fmaf(x0, c1.x, -z0 * s1.x), fmaf(x1, c1.y, -z1 * s1.y));
-            *p2 = pack_bf16x2(fmaf(z0, c2.x, x0 * s2.x), fmaf(z1, c2.y, x1 * s2.y));
+          bool q_ok = true;
+#pragma unroll
+          for (int bt = 0; bt < 2; ++bt) {
+            float2 c1[BATCH], c2[BATCH], s1[BATCH], s2[BATCH];
+#pragma unroll
+            for (int st = 0; st < BATCH; ++st) {
+              const int rr = wq * 32 + (bt * BATCH + st) * ROWS_PER_STEP + rsub;
+              const int pos = min(my_pb * BM + rr, p.S - 1);  // rows past S are zeros; any row's table is fine
+              const size_t trow = (static_cast<size_t>(b) * p.S + pos) * D;
+              c1[st] = *reinterpret_cast<const float2*>(p.cos + trow + d);
+              c2[st] = *reinterpret_cast<const float2*>(p.cos + trow + d2);
+              s1[st] = *reinterpret_cast<const float2*>(p.sin + trow + d);
+              s2[st] = *reinterpret_cast<const float2*>(p.sin + trow + d2);
+            }
+            if (bt == 0) q_ok = mbar_wait(&s.q_loaded[t], 0);
+            if (q_ok) {
+#pragma unroll
+              for (int st = 0; st < BATCH; ++st) {
+                const int rr = wq * 32 + (bt * BATCH + st) * ROWS_PER_STEP + rsub;
+                const uint32_t row = static_cast<uint32_t>(rr) * 128;
+                uint32_t* p1 = reinterpret_cast<uint32_t*>(qs + (d / 64) * BLOCK_BYTES + row +
+                                                           (((colb ^ (rr & 7)) << 4) | inb));
+                uint32_t* p2 = reinterpret_cast<uint32_t*>(qs + (d2 / 64) * BLOCK_BYTES + row +
+                                                           (((colb2 ^ (rr & 7)) << 4) | inb));
+                const uint32_t xa = *p1, za = *p2;
+                const float x0 = bf16lo(xa), x1 = bf16hi(xa), z0 = bf16lo(za), z1 = bf16hi(za);
+                *p1 = pack_bf16x2(fmaf(x0, c1[st].x, -z0 * s1[st].x), fmaf(x1, c1[st].y, -z1 * s1[st].y));
+                *p2 = pack_bf16x2(fmaf(z0, c2[st].x, x0 * s2[st].x), fmaf(z1, c2[st].y, x1 * s2[st].y));
+              }
+            }
           }
           fence_proxy_async_smem();
+        } else {
+          mbar_wait(&s.q_loaded[t], 0);
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&s.q_ready[t]);
@@ -357,47 +401,60 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
       for (int j = 0; j < n_kv; ++j) {
         if (!mbar_wait(&s.s_full[t], j & 1)) { ok = false; break; }
         tc_fence_after();
+        // S in two batches: the second half is in flight while the first half's
+        // max is taken
         uint32_t sr[4][32];
-#pragma unroll
-        for (int c = 0; c < 4; ++c) tmem_ld32(my_s + lane_off + c * 32, sr[c]);
-#pragma unroll
-        for (int c = 0; c < 4; ++c) tmem_ld_wait(sr[c]);
+        tmem_ld32(my_s + lane_off, sr[0]);
+        tmem_ld32(my_s + lane_off + 32, sr[1]);
+        tmem_ld_wait(sr[0]);
+        tmem_ld_wait(sr[1]);
+        tmem_ld32(my_s + lane_off + 64, sr[2]);
+        tmem_ld32(my_s + lane_off + 96, sr[3]);
         // v: raw scores (interior tiles: the scale is folded into the exponent's FMA)
         // or scaled + masked scores (tiles that touch the diagonal, the ragged end
         // or a mask, and any tile when scale <= 0)
         const int key0 = j * BN;
         const bool edge = (key0 + BN > p.S) || (p.causal && key0 + BN - 1 > my_pb * BM) ||
                           (mrow != nullptr) || !scale_pos;
-        float alpha = 1.f, rs = 0.f;
-        uint32_t pk[2][32];
+        float rs = 0.f;
         auto tile = [&](auto edge_c) {
           constexpr bool kEdge = decltype(edge_c)::value;
+          const int lim = p.causal ? min(p.S - 1, i) : p.S - 1;  // last visible key
           float v[BN];
-          if (!kEdge) {
+          auto fill = [&](int e0) {
 #pragma unroll
-            for (int e = 0; e < BN; ++e) v[e] = __uint_as_float(sr[e / 32][e % 32]);
-          } else {
-            const int lim = p.causal ? min(p.S - 1, i) : p.S - 1;  // last visible key
-#pragma unroll
-            for (int e = 0; e < BN; ++e) {
-              const int key = key0 + e;
-              float xv = __uint_as_float(sr[e / 32][e % 32]) * c_log2;
-              if (mrow != nullptr && key < p.S) xv = fmaf(mrow[key], 1.4426950408889634f, xv);
-              v[e] = (key <= lim) ? xv : -INFINITY;
+            for (int e = e0; e < e0 + BN / 2; ++e) {
+              if (!kEdge) {
+                v[e] = __uint_as_float(sr[e / 32][e % 32]);
+              } else {
+                const int key = key0 + e;
+                float xv = __uint_as_float(sr[e / 32][e % 32]) * c_log2;
+                if (mrow != nullptr && key < p.S) xv = fmaf(mrow[key], 1.4426950408889634f, xv);
+                v[e] = (key <= lim) ? xv : -INFINITY;
+              }
             }
-          }
+          };
           // row max: eight independent 3-input chains, then a small tree
           float mm[8];
+          fill(0);
 #pragma unroll
           for (int k = 0; k < 8; ++k) mm[k] = fmaxf(v[k], v[k + 8]);
 #pragma unroll
-          for (int e = 16; e < BN; e += 16)
+          for (int e = 16; e < BN / 2; e += 16)
+#pragma unroll
+            for (int k = 0; k < 8; ++k) mm[k] = fmax3f(mm[k], v[e + k], v[e + k + 8]);
+          tmem_ld_wait(sr[2]);
+          tmem_ld_wait(sr[3]);
+          fill(BN / 2);
+#pragma unroll
+          for (int e = BN / 2; e < BN; e += 16)
 #pragma unroll
             for (int k = 0; k < 8; ++k) mm[k] = fmax3f(mm[k], v[e + k], v[e + k + 8]);
           float mx = fmax3f(fmax3f(mm[0], mm[1], mm[2]), fmax3f(mm[3], mm[4], mm[5]),
                             fmaxf(mm[6], mm[7]));
           if (!kEdge) mx *= c_log2;
           // lazy reference: move only when the max grows by more than the threshold
+          float alpha = 1.f;
           if (mx > m_ref + kRescaleThreshold || (m_ref == -INFINITY && mx != -INFINITY)) {
             alpha = (m_ref == -INFINITY) ? 0.f : ex2_approx(m_ref - mx);
             m_ref = mx;
@@ -405,42 +462,50 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
           const float nref = (m_ref == -INFINITY) ? 0.f : -m_ref;
           const float cc = kEdge ? 1.f : c_log2;
           float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+          // P in two halves (keys 0-63, 64-127): the MMA warp starts O += P V on the
+          // first half while the second is being exponentiated
 #pragma unroll
-          for (int e = 0; e < BN; e += 2) {
-            float a0, a1, p0, p1;
-            ffma2(a0, a1, v[e], v[e + 1], cc, cc, nref, nref);  // exponent = v*c - m_ref
-            if (!kEdge && ((e / 2) % 8) < kPolyPairsOf8) {
-              exp2_poly2(p0, p1, a0, a1);
-            } else {
-              p0 = ex2_approx(a0);
-              p1 = ex2_approx(a1);
+          for (int h = 0; h < 2; ++h) {
+            uint32_t pk[32];
+#pragma unroll
+            for (int e = h * 64; e < h * 64 + 64; e += 2) {
+              float a0, a1, p0, p1;
+              ffma2(a0, a1, v[e], v[e + 1], cc, cc, nref, nref);  // exponent = v*c - m_ref
+              if (!kEdge && ((e / 2) % 8) < kPolyPairsOf8) {
+                exp2_poly2(p0, p1, a0, a1);
+              } else {
+                p0 = ex2_approx(a0);
+                p1 = ex2_approx(a1);
+              }
+              const int k = (e / 2) % 4;
+              fadd2(acc[2 * k], acc[2 * k + 1], acc[2 * k], acc[2 * k + 1], p0, p1);
+              pk[(e % 64) / 2] = pack_bf16x2(p0, p1);
             }
-            const int k = (e / 2) % 4;
-            fadd2(acc[2 * k], acc[2 * k + 1], acc[2 * k], acc[2 * k + 1], p0, p1);
-            pk[e / 64][(e % 64) / 2] = pack_bf16x2(p0, p1);
+            if (h == 0 && j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+              // O correction before any P of this tile is released (warp-collective
+              // TMEM access when any row of the warp needs it); PV_{j-1} has
+              // completed: its commit preceded this tile's S
+#pragma unroll
+              for (int c = 0; c < D / 32; ++c) {
+                uint32_t orr[32];
+                tmem_ld32(my_o + lane_off + c * 32, orr);
+                tmem_ld_wait(orr);
+#pragma unroll
+                for (int e = 0; e < 32; ++e) orr[e] = __float_as_uint(__uint_as_float(orr[e]) * alpha);
+                tmem_st32(my_o + lane_off + c * 32, orr);
+              }
+            }
+            tmem_st32(my_s + lane_off + h * 32, pk);
+            tmem_st_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(h == 0 ? &s.p_lo[t] : &s.p_hi[t]);
           }
           rs = ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
+          l_sum = fmaf(l_sum, alpha, rs);
         };
         if (edge) tile(std::true_type{});
         else tile(std::false_type{});
-        l_sum = fmaf(l_sum, alpha, rs);
-        // O correction (warp-collective TMEM access when any row of the warp needs it)
-        if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
-#pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
-            uint32_t orr[32];
-            tmem_ld32(my_o + lane_off + c * 32, orr);
-            tmem_ld_wait(orr);
-#pragma unroll
-            for (int e = 0; e < 32; ++e) orr[e] = __float_as_uint(__uint_as_float(orr[e]) * alpha);
-            tmem_st32(my_o + lane_off + c * 32, orr);
-          }
-        }
-        tmem_st32(my_s + lane_off, pk[0]);
-        tmem_st32(my_s + lane_off + 32, pk[1]);
-        tmem_st_wait();
-        tc_fence_before();
-        mbar_arrive(&s.p_full[t]);
       }
       // ---- epilogue: O / l -> bf16 -> out[b, i, head*D : head*D + D]
       if (ok && mbar_wait(&s.o_full[t], 0)) {
