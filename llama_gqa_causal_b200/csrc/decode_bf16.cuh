@@ -4,29 +4,42 @@
 // "GQA": several query heads share each K/V head, so one read of a K/V row
 // serves the whole group).
 //
-// Grid (split, kv_head x head_chunk, batch).  A CTA streams rows
-// [split*C, min((split+1)*C, len)) of one K/V head through a ring of TMA
-// stages (64 rows of K and V each, 128-byte swizzle) and computes, for up to
-// 8 query heads of the group at once, the partial softmax state (running max
-// m, sum l, un-normalised output o) over those rows.  Four consumer warps take
-// 16 rows of each stage:
-//   S^T[16 keys x 8 heads]  = K[16 x D] . Q'^T[D x 8]     (mma m16n8k16, K from
-//                                                          ldmatrix, Q' in regs)
-//   O^T[D x 8 heads]       += V^T[D x 16] . P^T[16 x 8]    (V^T by ldmatrix.trans,
+// Work is the flattened list of 256-row chunks of every sequence, where a
+// sequence is (batch entry, K/V head, chunk of <= 8 query heads of its group),
+// built on the device from cache_lens.  A persistent grid (one CTA per SM)
+// gives each CTA an even share of the chunks -- no two shares differ by more
+// than one chunk -- and each CTA streams its K/V rows through a ring of TMA
+// stages (64 rows of K and V each, 128-byte swizzle) without pausing at chunk
+// or sequence boundaries.  The query slice and its cos/sin row are brought by
+// bulk copy together with the first tile of each segment (a CTA's run of
+// tiles inside one sequence).
+//
+// Four consumer warps take 16 rows of each stage:
+//   S^T[16 keys x 8 heads]  = K[16 x D] . Q'^T[D x 8]    (mma m16n8k16; K by ldmatrix,
+//                                                          Q' in registers)
+//   O^T[D x 8 heads]       += V^T[D x 16] . P^T[16 x 8]   (V^T by ldmatrix.trans,
 //                                                          P^T by movmatrix)
-// so no tensor work is spent on padding when the group has 8 heads.  The
-// partial states of the four warps are merged in shared memory and written to
-// the workspace; decode_combine_kernel merges the splits with the
-// log-sum-exp identity and writes bf16 output.
+// so no tensor work is spent on padding when the group has 8 heads.  At the
+// end of a segment the warps merge their running (max, sum, output) and write
+// one partial: to the (batch, head) home slot when the segment starts at the
+// sequence's first row, otherwise to the CTA's own slot (only a CTA's first
+// segment can start inside a sequence).  decode_combine_kernel re-derives the
+// segment boundaries from the chunk counts and merges with the log-sum-exp
+// identity.
 #pragma once
 #include "common.cuh"
 
 namespace la {
 namespace dec {
-constexpr int TR = 64;      // cache rows per stage
-constexpr int NCW = 4;      // consumer warps (16 rows of a stage each)
-constexpr int NSTAGE = 3;   // ring depth
+constexpr int TR = 64;           // cache rows per stage
+constexpr int CH = 256;          // rows per work chunk (granule of the even split)
+constexpr int NCW = 4;           // consumer warps (16 rows of a stage each)
+constexpr int NSTAGE = 5;        // ring depth
 constexpr int THREADS = (NCW + 1) * 32;
+constexpr int MAX_BATCH = 4096;  // per-batch chunk prefix lives in shared memory
+constexpr int MAX_CTAS = 256;    // persistent grid size cap (one CTA per SM)
+// floats per partial row: D outputs, then max and sum; padded to 16 bytes
+__host__ __device__ constexpr int part_stride(int d) { return d + 4; }
 }  // namespace dec
 
 struct DecodeParams {
@@ -34,20 +47,36 @@ struct DecodeParams {
   const float* cos;        // [b, D] or null
   const float* sin;
   const int* lens;         // [b]
-  float* ws_o;             // [b, H, n_splits, D]
-  float* ws_ml;            // [b, H, n_splits, 2]
-  int bsz, H, Hkv, L, group, hchunks, split_rows, n_splits;
+  float* ws_home;          // [b, H, D + 4]: partial of the segment at a sequence's start
+  float* ws_cta;           // [MAX_CTAS, 8, D + 4]: partial of a CTA's mid-sequence segment
+  int bsz, H, Hkv, L, group, hchunks;
   float scale_log2;        // scale * log2(e)
+};
+
+// Per-stage description of the tile, written by the producer before it arms
+// the stage's barrier.
+struct DecTileMeta {
+  int b, kvh, hc;
+  int nvalid;      // rows of the tile below the sequence length (1..TR)
+  int seg_start;   // first tile of a segment: consumers reset and read q
+  int seg_end;     // last tile of a segment: consumers merge and write a partial
+  int home;        // the segment starts at row 0 of its sequence
+  int last;        // the CTA's final tile
 };
 
 template <int D>
 struct DecSmem {
   alignas(1024) __nv_bfloat16 k[dec::NSTAGE][dec::TR * D];
   alignas(1024) __nv_bfloat16 v[dec::NSTAGE][dec::TR * D];
+  alignas(16) __nv_bfloat16 qv[dec::NSTAGE][8 * D];  // query slice at segment starts
+  alignas(16) float cs[dec::NSTAGE][2 * D];            // cos row, sin row at segment starts
+  DecTileMeta meta[dec::NSTAGE];
   uint64_t full[dec::NSTAGE];
   uint64_t empty[dec::NSTAGE];
+  float red_o[dec::NCW][8][D + 4];  // +4 spreads the merge's rows over the banks
   float red_m[dec::NCW][8];
   float red_l[dec::NCW][8];
+  int chunk_prefix[dec::MAX_BATCH + 1];  // chunks per sequence of batch entries < b
 };
 
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
@@ -77,9 +106,29 @@ __device__ __forceinline__ void mma_bf16_16816(float (&c)[4], uint32_t a0, uint3
       : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
+// Untiled bulk copy global -> shared completing on an mbarrier
+// (both addresses 16-byte aligned, size a multiple of 16).
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ int clamp_len(int len, int L) { return len < 0 ? 0 : (len > L ? L : len); }
+
+// Even split of n chunks over g CTAs: CTA i owns chunks [share_start(i), share_start(i + 1)).
+__device__ __forceinline__ long long share_start(long long i, long long n, long long g) {
+  return (i * n) / g;
+}
+// The CTA whose share holds chunk x: the largest i with share_start(i) <= x.
+__device__ __forceinline__ long long share_owner(long long x, long long n, long long g) {
+  return ((x + 1) * g + n - 1) / n - 1;
+}
 
 template <int D>
-__global__ void __launch_bounds__(dec::THREADS) decode_bf16_kernel(
+__global__ void __launch_bounds__(dec::THREADS, 1) decode_bf16_kernel(
     const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
     DecodeParams p) {
   using namespace dec;
@@ -91,18 +140,16 @@ __global__ void __launch_bounds__(dec::THREADS) decode_bf16_kernel(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int split = blockIdx.x;
-  const int kvh = blockIdx.y / p.hchunks, hc = blockIdx.y - kvh * p.hchunks;
-  const int b = blockIdx.z;
-  int len = p.lens[b];
-  len = len < 0 ? 0 : (len > p.L ? p.L : len);
-  const int start = split * p.split_rows;
-  if (start >= len) return;  // uniform across the block, before any barrier
-  const int rows = min(p.split_rows, len - start);
-  const int nT = (rows + TR - 1) / TR;
-  const int bh = b * p.Hkv + kvh;
+  const int per_b = p.Hkv * p.hchunks;  // sequences per batch entry
 
+  // ---- chunk counts per batch entry, prefix-summed (identical in every CTA)
   if (threadIdx.x == 0) {
+    int acc = 0;
+    for (int b = 0; b < p.bsz; ++b) {
+      s.chunk_prefix[b] = acc;
+      acc += (clamp_len(p.lens[b], p.L) + CH - 1) / CH;
+    }
+    s.chunk_prefix[p.bsz] = acc;
     for (int i = 0; i < NSTAGE; ++i) {
       mbar_init(&s.full[i], 1);
       mbar_init(&s.empty[i], NCW);
@@ -110,79 +157,129 @@ __global__ void __launch_bounds__(dec::THREADS) decode_bf16_kernel(
     fence_mbar_init();
   }
   __syncthreads();
+  // the combine kernel may be scheduled now; it waits for this grid to finish
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  const long long n_chunks = static_cast<long long>(s.chunk_prefix[p.bsz]) * per_b;
+  const long long x0 = share_start(blockIdx.x, n_chunks, gridDim.x);
+  const long long x1 = share_start(blockIdx.x + 1, n_chunks, gridDim.x);
+  if (x0 >= x1) return;  // uniform across the CTA: no share
 
   if (warp == NCW) {  // ---------------------------------------------- TMA producer
-    if (lane == 0) {
+    if (elect_one()) {
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
-      int issued = 0;
-      for (int it = 0; it < nT; ++it) {
-        const int st = it % NSTAGE;
-        if (it >= NSTAGE && !mbar_wait(&s.empty[st], ((it / NSTAGE) - 1) & 1)) break;
-        mbar_arrive_expect_tx(&s.full[st], 2u * TR * D * 2u);
-#pragma unroll
-        for (int cb = 0; cb < CB; ++cb) {
-          tma_load_3d(&s.k[st][cb * TR * 64], &tm_k, &s.full[st], cb * 64, start + it * TR, bh);
-          tma_load_3d(&s.v[st][cb * TR * 64], &tm_v, &s.full[st], cb * 64, start + it * TR, bh);
-        }
-        issued = it + 1;
-      }
-      // never leave with copies in flight: wait for every issued stage to land
-      for (int it = max(0, issued - NSTAGE); it < issued; ++it)
-        if (!mbar_wait(&s.full[it % NSTAGE], (it / NSTAGE) & 1)) break;
     }
+    __syncwarp();
+    int b = 0;
+    int it = 0;  // tiles issued
+    bool ok = true;
+    bool home = false;
+    for (long long x = x0; x < x1 && ok; ++x) {
+      // global chunk x -> batch entry b, sequence (kvh, hc) within b, chunk c
+      while (static_cast<long long>(s.chunk_prefix[b + 1]) * per_b <= x) ++b;
+      const int nch_b = s.chunk_prefix[b + 1] - s.chunk_prefix[b];
+      const long long xb = x - static_cast<long long>(s.chunk_prefix[b]) * per_b;
+      const int seq = static_cast<int>(xb / nch_b);
+      const int c = static_cast<int>(xb - static_cast<long long>(seq) * nch_b);
+      const int kvh = seq / p.hchunks, hc = seq - kvh * p.hchunks;
+      const int len = clamp_len(p.lens[b], p.L);
+      const bool first_chunk_of_seg = (x == x0) || (c == 0);
+      const bool last_chunk_of_seg = (x + 1 == x1) || (c + 1 == nch_b);
+      if (first_chunk_of_seg) home = (c == 0);
+      const int row_end = min(len, (c + 1) * CH);
+      for (int row0 = c * CH; row0 < row_end; row0 += TR, ++it) {
+        const int st = it % NSTAGE;
+        if (it >= NSTAGE && !mbar_wait(&s.empty[st], ((it / NSTAGE) - 1) & 1)) {
+          ok = false;
+          break;
+        }
+        const bool seg_start = first_chunk_of_seg && row0 == c * CH;
+        const bool tile_last_of_chunk = row0 + TR >= row_end;
+        if (elect_one()) {
+          DecTileMeta& m = s.meta[st];
+          m.b = b;
+          m.kvh = kvh;
+          m.hc = hc;
+          m.nvalid = min(TR, row_end - row0);
+          m.seg_start = seg_start;
+          m.seg_end = last_chunk_of_seg && tile_last_of_chunk;
+          m.home = home;
+          m.last = (x + 1 == x1) && tile_last_of_chunk;
+          const int nh = min(8, p.group - hc * 8);
+          uint32_t bytes = 2u * TR * D * 2u;
+          if (seg_start) bytes += nh * D * 2u + (p.cos != nullptr ? 2u * D * 4u : 0u);
+          mbar_arrive_expect_tx(&s.full[st], bytes);
+          const int bh = b * p.Hkv + kvh;
+#pragma unroll
+          for (int cb = 0; cb < CB; ++cb) {
+            tma_load_3d(&s.k[st][cb * TR * 64], &tm_k, &s.full[st], cb * 64, row0, bh);
+            tma_load_3d(&s.v[st][cb * TR * 64], &tm_v, &s.full[st], cb * 64, row0, bh);
+          }
+          if (seg_start) {
+            bulk_load(&s.qv[st][0], p.q + (static_cast<size_t>(b) * p.H + kvh * p.group + hc * 8) * D,
+                      nh * D * 2u, &s.full[st]);
+            if (p.cos != nullptr) {
+              bulk_load(&s.cs[st][0], p.cos + static_cast<size_t>(b) * D, D * 4u, &s.full[st]);
+              bulk_load(&s.cs[st][D], p.sin + static_cast<size_t>(b) * D, D * 4u, &s.full[st]);
+            }
+          }
+        }
+        __syncwarp();
+      }
+    }
+    // never leave with copies in flight: wait for the last issued stages to land
+    for (int i = max(0, it - NSTAGE); i < it; ++i)
+      if (!mbar_wait(&s.full[i % NSTAGE], (i / NSTAGE) & 1)) break;
     return;
   }
 
   // ------------------------------------------------------------------ consumers
   const int g = lane >> 2, t = lane & 3;
-  const int hq = hc * 8 + g;  // query head within the group held by this lane's B columns
-  const bool hvalid = hq < p.group;
-  // Q' fragments: lane holds head hq, dims kk*16 + 2t + {0, 1, 8, 9}.  The
-  // rotation partner of dim d is d +- D/2, i.e. k-step kk +- D/32, same lane.
+  const int mat = lane >> 3, r8 = lane & 7;
   uint32_t qf[KSTEPS][2];
-  {
-    float qx[KSTEPS][4];
-    const __nv_bfloat16* qr = p.q + (static_cast<size_t>(b) * p.H + kvh * p.group + hq) * D;
-#pragma unroll
-    for (int kk = 0; kk < KSTEPS; ++kk)
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int d = kk * 16 + 2 * t + (j < 2 ? j : j + 6);
-        qx[kk][j] = hvalid ? __bfloat162float(qr[d]) : 0.f;
-      }
-#pragma unroll
-    for (int kk = 0; kk < KSTEPS; ++kk) {
-      float y[4];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        y[j] = qx[kk][j];
-        if (p.cos != nullptr) {
-          const int d = kk * 16 + 2 * t + (j < 2 ? j : j + 6);
-          const float c = p.cos[static_cast<size_t>(b) * D + d];
-          const float sn = p.sin[static_cast<size_t>(b) * D + d];
-          const float rot = (kk < KSTEPS / 2) ? -qx[kk + KSTEPS / 2][j] : qx[kk - KSTEPS / 2][j];
-          y[j] = fmaf(qx[kk][j], c, rot * sn);
-        }
-      }
-      qf[kk][0] = pack_bf16x2(y[0], y[1]);
-      qf[kk][1] = pack_bf16x2(y[2], y[3]);
-    }
-  }
-
-  float m_run[2] = {-INFINITY, -INFINITY};
-  float l_run[2] = {0.f, 0.f};
+  float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.f, 0.f};
   float o[KSTEPS][4];
 #pragma unroll
   for (int mt = 0; mt < KSTEPS; ++mt) o[mt][0] = o[mt][1] = o[mt][2] = o[mt][3] = 0.f;
-
-  const int mat = lane >> 3, r8 = lane & 7;
-  bool ok = true;
-  for (int it = 0; it < nT; ++it) {
+#pragma unroll
+  for (int kk = 0; kk < KSTEPS; ++kk) qf[kk][0] = qf[kk][1] = 0u;
+  for (int it = 0;; ++it) {
     const int st = it % NSTAGE;
-    if (!mbar_wait(&s.full[st], (it / NSTAGE) & 1)) { ok = false; break; }
-    const int key0 = start + it * TR + warp * 16;
-    const int nvalid = min(16, len - key0);
+    if (!mbar_wait(&s.full[st], (it / NSTAGE) & 1)) break;
+    const DecTileMeta m = s.meta[st];
+    if (m.seg_start) {
+      m_run[0] = m_run[1] = -INFINITY;
+      l_run[0] = l_run[1] = 0.f;
+#pragma unroll
+      for (int mt = 0; mt < KSTEPS; ++mt) o[mt][0] = o[mt][1] = o[mt][2] = o[mt][3] = 0.f;
+      // Q' fragments: lane holds head g of the chunk, dims kk*16 + 2t + {0, 1, 8, 9}.
+      // The rotation partner of dim d is d +- D/2, i.e. k-step kk +- D/32, same lane.
+      const bool hvalid = m.hc * 8 + g < p.group;
+      float qx[KSTEPS][4];
+#pragma unroll
+      for (int kk = 0; kk < KSTEPS; ++kk)
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) {
+          const int d = kk * 16 + 2 * t + (jj < 2 ? jj : jj + 6);
+          qx[kk][jj] = hvalid ? __bfloat162float(s.qv[st][g * D + d]) : 0.f;
+        }
+#pragma unroll
+      for (int kk = 0; kk < KSTEPS; ++kk) {
+        float y[4];
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) {
+          y[jj] = qx[kk][jj];
+          if (p.cos != nullptr) {
+            const int d = kk * 16 + 2 * t + (jj < 2 ? jj : jj + 6);
+            const float rot = (kk < KSTEPS / 2) ? -qx[kk + KSTEPS / 2][jj] : qx[kk - KSTEPS / 2][jj];
+            y[jj] = fmaf(qx[kk][jj], s.cs[st][d], rot * s.cs[st][D + d]);
+          }
+        }
+        qf[kk][0] = pack_bf16x2(y[0], y[1]);
+        qf[kk][1] = pack_bf16x2(y[2], y[3]);
+      }
+    }
+    const int nvalid = min(16, m.nvalid - warp * 16);
     const uint32_t kbase = smem_u32(&s.k[st][0]);
     const uint32_t vbase = smem_u32(&s.v[st][0]);
     if (nvalid > 0) {
@@ -193,8 +290,8 @@ __global__ void __launch_bounds__(dec::THREADS) decode_bf16_kernel(
         for (int idx = lane; idx < (16 - nvalid) * CB * 8; idx += 32) {
           const int rr = warp * 16 + nvalid + idx / (CB * 8);
           const int rem = idx % (CB * 8);
-          *reinterpret_cast<uint4*>(vb + (rem / 8) * STAGE_BLOCK_BYTES +
-                                    sw128_offset(rr, rem % 8)) = make_uint4(0, 0, 0, 0);
+          *reinterpret_cast<uint4*>(vb + (rem / 8) * STAGE_BLOCK_BYTES + sw128_offset(rr, rem % 8)) =
+              make_uint4(0, 0, 0, 0);
         }
         fence_proxy_async_smem();
         __syncwarp();
@@ -206,8 +303,8 @@ __global__ void __launch_bounds__(dec::THREADS) decode_bf16_kernel(
       for (int kk = 0; kk < KSTEPS; ++kk) {
         const int col = kk * 16 + (mat >> 1) * 8;
         uint32_t a0, a1, a2, a3;
-        ldsm_x4(kbase + (col / 64) * STAGE_BLOCK_BYTES + sw128_offset(krow, (col % 64) / 8), a0,
-                a1, a2, a3);
+        ldsm_x4(kbase + (col / 64) * STAGE_BLOCK_BYTES + sw128_offset(krow, (col % 64) / 8), a0, a1,
+                a2, a3);
         mma_bf16_16816(sc, a0, a1, a2, a3, qf[kk][0], qf[kk][1]);
       }
       // sc[0]=(key g, head 2t) sc[1]=(key g, head 2t+1) sc[2]=(key g+8, 2t) sc[3]=(key g+8, 2t+1)
@@ -224,7 +321,7 @@ __global__ void __launch_bounds__(dec::THREADS) decode_bf16_kernel(
         mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
         mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
         mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
-        const float m_new = fmaxf(m_run[h], mx);  // finite: key0 < len is valid
+        const float m_new = fmaxf(m_run[h], mx);  // finite: this warp has a valid key
         alpha[h] = (m_run[h] == -INFINITY) ? 0.f : ex2_approx(m_run[h] - m_new);
         pr[h] = ex2_approx(x[h] - m_new);
         pr[h + 2] = ex2_approx(x[h + 2] - m_new);
@@ -247,95 +344,135 @@ __global__ void __launch_bounds__(dec::THREADS) decode_bf16_kernel(
       for (int mt = 0; mt < KSTEPS; ++mt) {
         const int col = mt * 16 + (mat & 1) * 8;
         uint32_t a0, a1, a2, a3;
-        ldsm_x4_t(vbase + (col / 64) * STAGE_BLOCK_BYTES + sw128_offset(vrow, (col % 64) / 8),
-                  a0, a1, a2, a3);
+        ldsm_x4_t(vbase + (col / 64) * STAGE_BLOCK_BYTES + sw128_offset(vrow, (col % 64) / 8), a0,
+                  a1, a2, a3);
         mma_bf16_16816(o[mt], a0, a1, a2, a3, pb0, pb1);
       }
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(&s.empty[st]);
-  }
 
-  // ---- merge the four warps' partial states (stage memory reused as scratch)
+    if (m.seg_end) {
+      // ---- merge the four warps' partial states, write the segment's partial
+      float lr[2] = {l_run[0], l_run[1]};
 #pragma unroll
-  for (int h = 0; h < 2; ++h) {
-    l_run[h] += __shfl_xor_sync(0xffffffffu, l_run[h], 4);
-    l_run[h] += __shfl_xor_sync(0xffffffffu, l_run[h], 8);
-    l_run[h] += __shfl_xor_sync(0xffffffffu, l_run[h], 16);
-  }
-  named_bar_sync(1, NCW * 32);  // every warp is done reading the stages
-  if (!ok) return;               // a wait ran out: leave without writing
-  float* red_o = reinterpret_cast<float*>(&s.k[0][0]);  // [NCW][8][D]
-  if (g == 0) {
-    s.red_m[warp][2 * t] = m_run[0];
-    s.red_m[warp][2 * t + 1] = m_run[1];
-    s.red_l[warp][2 * t] = l_run[0];
-    s.red_l[warp][2 * t + 1] = l_run[1];
-  }
-#pragma unroll
-  for (int mt = 0; mt < KSTEPS; ++mt) {
-    red_o[(warp * 8 + 2 * t) * D + mt * 16 + g] = o[mt][0];
-    red_o[(warp * 8 + 2 * t + 1) * D + mt * 16 + g] = o[mt][1];
-    red_o[(warp * 8 + 2 * t) * D + mt * 16 + g + 8] = o[mt][2];
-    red_o[(warp * 8 + 2 * t + 1) * D + mt * 16 + g + 8] = o[mt][3];
-  }
-  named_bar_sync(1, NCW * 32);
-  {
-    constexpr int PER = D / 16;  // dims per thread: 128 threads cover 8 heads x D
-    const int tid = threadIdx.x;
-    const int hh = tid >> 4;
-    const int d0 = (tid & 15) * PER;
-    const int hq2 = hc * 8 + hh;
-    if (hq2 < p.group) {
-      float mstar = -INFINITY;
-#pragma unroll
-      for (int w = 0; w < NCW; ++w) mstar = fmaxf(mstar, s.red_m[w][hh]);
-      float f[NCW], lsum = 0.f;
-#pragma unroll
-      for (int w = 0; w < NCW; ++w) {
-        const float mw = s.red_m[w][hh];
-        f[w] = (mw == -INFINITY) ? 0.f : ex2_approx(mw - mstar);
-        lsum = fmaf(f[w], s.red_l[w][hh], lsum);
+      for (int h = 0; h < 2; ++h) {
+        lr[h] += __shfl_xor_sync(0xffffffffu, lr[h], 4);
+        lr[h] += __shfl_xor_sync(0xffffffffu, lr[h], 8);
+        lr[h] += __shfl_xor_sync(0xffffffffu, lr[h], 16);
       }
-      const int head = kvh * p.group + hq2;
-      const size_t slot = (static_cast<size_t>(b) * p.H + head) * p.n_splits + split;
-      float* dst = p.ws_o + slot * D + d0;
-#pragma unroll
-      for (int i = 0; i < PER; ++i) {
-        float acc = 0.f;
-#pragma unroll
-        for (int w = 0; w < NCW; ++w) acc = fmaf(f[w], red_o[(w * 8 + hh) * D + d0 + i], acc);
-        dst[i] = acc;
+      if (g == 0) {
+        s.red_m[warp][2 * t] = m_run[0];
+        s.red_m[warp][2 * t + 1] = m_run[1];
+        s.red_l[warp][2 * t] = lr[0];
+        s.red_l[warp][2 * t + 1] = lr[1];
       }
-      if ((tid & 15) == 0) {
-        p.ws_ml[slot * 2] = mstar;
-        p.ws_ml[slot * 2 + 1] = lsum;
+#pragma unroll
+      for (int mt = 0; mt < KSTEPS; ++mt) {
+        s.red_o[warp][2 * t][mt * 16 + g] = o[mt][0];
+        s.red_o[warp][2 * t + 1][mt * 16 + g] = o[mt][1];
+        s.red_o[warp][2 * t][mt * 16 + g + 8] = o[mt][2];
+        s.red_o[warp][2 * t + 1][mt * 16 + g + 8] = o[mt][3];
       }
+      named_bar_sync(1, NCW * 32);
+      {
+        constexpr int PER = D / 16;  // dims per thread: 128 threads cover 8 heads x D
+        const int tid = threadIdx.x;
+        const int hh = tid >> 4;
+        const int d0 = (tid & 15) * PER;
+        if (m.hc * 8 + hh < p.group) {
+          float mstar = -INFINITY;
+#pragma unroll
+          for (int w = 0; w < NCW; ++w) mstar = fmaxf(mstar, s.red_m[w][hh]);
+          float f[NCW], lsum = 0.f;
+#pragma unroll
+          for (int w = 0; w < NCW; ++w) {
+            const float mw = s.red_m[w][hh];
+            f[w] = (mw == -INFINITY) ? 0.f : ex2_approx(mw - mstar);
+            lsum = fmaf(f[w], s.red_l[w][hh], lsum);
+          }
+          const int head = m.kvh * p.group + m.hc * 8 + hh;
+          float* dst = m.home
+              ? p.ws_home + (static_cast<size_t>(m.b) * p.H + head) * part_stride(D)
+              : p.ws_cta + (static_cast<size_t>(blockIdx.x) * 8 + hh) * part_stride(D);
+#pragma unroll
+          for (int i = 0; i < PER; i += 4) {
+            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+            for (int w = 0; w < NCW; ++w) {
+              acc.x = fmaf(f[w], s.red_o[w][hh][d0 + i], acc.x);
+              acc.y = fmaf(f[w], s.red_o[w][hh][d0 + i + 1], acc.y);
+              acc.z = fmaf(f[w], s.red_o[w][hh][d0 + i + 2], acc.z);
+              acc.w = fmaf(f[w], s.red_o[w][hh][d0 + i + 3], acc.w);
+            }
+            *reinterpret_cast<float4*>(dst + d0 + i) = acc;
+          }
+          if ((tid & 15) == 0) {
+            dst[D] = mstar;
+            dst[D + 1] = lsum;
+          }
+        }
+      }
+      named_bar_sync(1, NCW * 32);  // red_* are reused by the next segment
     }
+    if (m.last) break;
   }
 }
 
-// Merge the per-split partial states of one (b, head):
+// Merge the partials of one (b, head).  Its sequence's segments start at the
+// sequence's first chunk (home slot) and at every chunk where some CTA's share
+// begins inside the sequence (that CTA's own slot).
 //   m* = max_s m_s,  l = sum_s l_s 2^(m_s - m*),  o = sum_s o_s 2^(m_s - m*) / l.
 template <int D>
-__global__ void __launch_bounds__(D) decode_combine_kernel(const float* __restrict__ ws_o,
-                                                           const float* __restrict__ ws_ml,
+__global__ void __launch_bounds__(D) decode_combine_kernel(const float* __restrict__ ws_home,
+                                                           const float* __restrict__ ws_cta,
                                                            const int* __restrict__ lens,
                                                            __nv_bfloat16* __restrict__ out,
-                                                           int H, int L, int split_rows,
-                                                           int n_splits) {
+                                                           int bsz, int H, int Hkv, int L,
+                                                           int group, int hchunks, int n_ctas) {
+  // the split kernel's writes are visible after this (programmatic dependent launch)
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const int h = blockIdx.x, b = blockIdx.y, d = threadIdx.x;
-  int len = lens[b];
-  len = len < 0 ? 0 : (len > L ? L : len);
-  const int n = (len + split_rows - 1) / split_rows;
-  const size_t slot0 = (static_cast<size_t>(b) * H + h) * n_splits;
-  float mstar = -INFINITY;
-  for (int s = 0; s < n; ++s) mstar = fmaxf(mstar, ws_ml[(slot0 + s) * 2]);
-  float lsum = 0.f, acc = 0.f;
-  for (int s = 0; s < n; ++s) {
-    const float f = ex2_approx(ws_ml[(slot0 + s) * 2] - mstar);
-    lsum = fmaf(f, ws_ml[(slot0 + s) * 2 + 1], lsum);
-    acc = fmaf(f, ws_o[(slot0 + s) * D + d], acc);
+  __shared__ long long sh_prefix_b, sh_total;
+  if (d == 0) {
+    long long acc = 0, pre = 0;
+    for (int i = 0; i < bsz; ++i) {
+      if (i == b) pre = acc;
+      acc += (clamp_len(lens[i], L) + dec::CH - 1) / dec::CH;
+    }
+    sh_prefix_b = pre;
+    sh_total = acc;
+  }
+  __syncthreads();
+  const int per_b = Hkv * hchunks;
+  const int nch = (clamp_len(lens[b], L) + dec::CH - 1) / dec::CH;
+  const int kvh = h / group, hq = h - kvh * group, hc = hq / 8, hh = hq % 8;
+  const long long n_chunks = sh_total * per_b;
+  const long long G = n_ctas;
+  const long long P = sh_prefix_b * per_b + static_cast<long long>(kvh * hchunks + hc) * nch;
+  float mstar = -INFINITY, lsum = 0.f, acc = 0.f;
+  auto add = [&](const float* part) {
+    const float mc = part[D], lc = part[D + 1];
+    const float m_new = fmaxf(mstar, mc);
+    const float fo = (mstar == -INFINITY) ? 0.f : ex2_approx(mstar - m_new);
+    const float fc = ex2_approx(mc - m_new);
+    lsum = lsum * fo + lc * fc;
+    acc = acc * fo + part[d] * fc;
+    mstar = m_new;
+  };
+  if (nch > 0) {
+    add(ws_home + (static_cast<size_t>(b) * H + h) * dec::part_stride(D));
+    // CTA shares that begin strictly inside [P, P + nch); equal starts mean empty
+    // shares, and the owner of a start is the last CTA with that start
+    long long last_start = P;
+    for (long long gi = share_owner(P, n_chunks, G) + 1; gi < G; ++gi) {
+      const long long st = share_start(gi, n_chunks, G);
+      if (st >= P + nch) break;
+      if (st == last_start) continue;
+      last_start = st;
+      const long long owner = share_owner(st, n_chunks, G);
+      add(ws_cta + (static_cast<size_t>(owner) * 8 + hh) * dec::part_stride(D));
+    }
   }
   const float r = (lsum > 0.f) ? acc / lsum : 0.f;
   out[(static_cast<size_t>(b) * H + h) * D + d] = __float2bfloat16_rn(r);

@@ -19,7 +19,6 @@
 namespace {
 
 constexpr int kAbiVersion = 100;
-constexpr int kDecodeSplitRows = 512;  // cache rows per decode CTA (multiple of dec::TR)
 
 // ---------------------------------------------------------------- host helpers
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -95,10 +94,6 @@ int check_common(int bsz, int n_heads, int n_kv_heads, int head_dim, int dtype,
   return LLAMA_OK;
 }
 
-int decode_splits(int max_cache_len) {
-  return (max_cache_len + kDecodeSplitRows - 1) / kDecodeSplitRows;
-}
-
 // ---------------------------------------------------------------- prefill dispatch
 template <int D>
 int prefill_bf16(const void* q, const void* k, const void* v, const float* cos, const float* sin,
@@ -172,11 +167,22 @@ int attn_fp32(const float* q, const float* k, const float* v, const float* cos, 
   return launch_status();
 }
 
+int sm_count() {
+  static int count[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+  if (count[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    count[dev] = n;
+  }
+  return count[dev];
+}
+
 template <int D>
 int decode_bf16(const void* q, const void* kc, const void* vc, const int* lens, const float* cos,
                 const float* sin, int bsz, int H, int Hkv, int L, float scale, void* out,
                 void* workspace, cudaStream_t st) {
-  const int n_splits = decode_splits(L);
   CUtensorMap tk, tv;
   const cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(L),
                               static_cast<cuuint64_t>(bsz) * Hkv};
@@ -184,29 +190,48 @@ int decode_bf16(const void* q, const void* kc, const void* vc, const int* lens, 
   const cuuint32_t box[3] = {64, static_cast<cuuint32_t>(la::dec::TR), 1};
   if (!make_map(&tk, kc, 3, dims, strides, box)) return LLAMA_ERR_CUDA;
   if (!make_map(&tv, vc, 3, dims, strides, box)) return LLAMA_ERR_CUDA;
+  const int n_ctas = std::min(sm_count(), la::dec::MAX_CTAS);
+  if (n_ctas <= 0) return LLAMA_ERR_CUDA;
   la::DecodeParams p;
   p.q = static_cast<const __nv_bfloat16*>(q);
   p.cos = cos;
   p.sin = sin;
   p.lens = lens;
-  p.ws_o = static_cast<float*>(workspace);
-  p.ws_ml = p.ws_o + static_cast<size_t>(bsz) * H * n_splits * D;
+  p.ws_home = static_cast<float*>(workspace);
+  p.ws_cta = p.ws_home + static_cast<size_t>(bsz) * H * la::dec::part_stride(D);
   p.bsz = bsz;
   p.H = H;
   p.Hkv = Hkv;
   p.L = L;
   p.group = H / Hkv;
   p.hchunks = (p.group + 7) / 8;
-  p.split_rows = kDecodeSplitRows;
-  p.n_splits = n_splits;
   p.scale_log2 = scale * 1.4426950408889634f;
   const size_t smem = sizeof(la::DecSmem<D>) + 1024;
   if (!ensure_smem_attr<la::decode_bf16_kernel<D>>(smem)) return LLAMA_ERR_CUDA;
-  dim3 grid(n_splits, Hkv * p.hchunks, bsz);
-  la::decode_bf16_kernel<D><<<grid, la::dec::THREADS, smem, st>>>(tk, tv, p);
+  la::decode_bf16_kernel<D><<<n_ctas, la::dec::THREADS, smem, st>>>(tk, tv, p);
   if (int e = launch_status()) return e;
-  la::decode_combine_kernel<D><<<dim3(H, bsz), D, 0, st>>>(
-      p.ws_o, p.ws_ml, lens, static_cast<__nv_bfloat16*>(out), H, L, kDecodeSplitRows, n_splits);
+  // the combine launches as a programmatic dependent of the split kernel: its
+  // blocks are scheduled while the split kernel drains and wait on the device
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(H, bsz);
+  cfg.blockDim = dim3(D);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const float* home = p.ws_home;
+  const float* ctas = p.ws_cta;
+  __nv_bfloat16* o = static_cast<__nv_bfloat16*>(out);
+  int group = p.group, hchunks = p.hchunks;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, la::decode_combine_kernel<D>, home, ctas, lens, o,
+                                           bsz, H, Hkv, L, group, hchunks, n_ctas);
+  if (e != cudaSuccess) {
+    fprintf(stderr, "llama_attn: combine launch failed: %s\n", cudaGetErrorString(e));
+    return LLAMA_ERR_CUDA;
+  }
   return launch_status();
 }
 
@@ -314,8 +339,9 @@ int llama_attn_prefill(const void* q, const void* k, const void* v, const float*
 
 size_t llama_attn_decode_workspace_bytes(int bsz, int n_heads, int max_cache_len, int head_dim) {
   if (bsz < 1 || n_heads < 1 || max_cache_len < 1 || head_dim < 1) return 0;
-  const size_t slots = static_cast<size_t>(bsz) * n_heads * decode_splits(max_cache_len);
-  return slots * (static_cast<size_t>(head_dim) + 2) * sizeof(float);
+  // one partial per (batch, head) plus one per (CTA, head of an 8-head chunk)
+  const size_t rows = static_cast<size_t>(bsz) * n_heads + static_cast<size_t>(la::dec::MAX_CTAS) * 8;
+  return rows * la::dec::part_stride(head_dim) * sizeof(float);
 }
 
 int llama_attn_decode(const void* q, const void* k_cache, const void* v_cache,
@@ -332,6 +358,7 @@ int llama_attn_decode(const void* q, const void* k_cache, const void* v_cache,
     return LLAMA_ERR_INVALID_ARG;
   cudaStream_t st = as_stream(cuda_stream);
   if (dtype == LLAMA_DT_BF16) {
+    if (bsz > la::dec::MAX_BATCH) return LLAMA_ERR_UNSUPPORTED;
     const size_t need = llama_attn_decode_workspace_bytes(bsz, n_heads, max_cache_len, head_dim);
     if (workspace == nullptr || workspace_bytes < need) return LLAMA_ERR_INVALID_ARG;
     if (head_dim == 128)

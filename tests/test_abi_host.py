@@ -55,9 +55,11 @@ def test_workspace_sizes(lib):
     assert lib.llama_attn_prefill_workspace_bytes(1, 64, 8, 8192, 128, 1, 1) == 8192 * 8 * 128 * 2
     assert lib.llama_attn_prefill_workspace_bytes(1, 64, 8, 8192, 128, 1, 0) == 0
     assert lib.llama_attn_prefill_workspace_bytes(1, 4, 2, 64, 64, 0, 1) == 0
-    # decode: (D + 2) floats per (b, head, split of 512 rows)
-    assert lib.llama_attn_decode_workspace_bytes(32, 64, 4096, 128) == 32 * 64 * 8 * 130 * 4
-    assert lib.llama_attn_decode_workspace_bytes(2, 4, 513, 64) == 2 * 4 * 2 * 66 * 4
+    # decode: one partial row of D + 4 floats per (b, head) and per (CTA, head of
+    # an 8-head chunk) for up to 256 CTAs; independent of the cache length
+    assert lib.llama_attn_decode_workspace_bytes(32, 64, 4096, 128) == (32 * 64 + 256 * 8) * 132 * 4
+    assert lib.llama_attn_decode_workspace_bytes(2, 4, 513, 64) == (2 * 4 + 256 * 8) * 68 * 4
+    assert lib.llama_attn_decode_workspace_bytes(2, 4, 1 << 20, 64) == (2 * 4 + 256 * 8) * 68 * 4
     assert lib.llama_attn_decode_workspace_bytes(0, 4, 513, 64) == 0
 
 
@@ -134,8 +136,8 @@ def test_rope_table_rejects(lib, args):
 
 
 def test_decode_noalloc_refuses_what_its_static_scratch_cannot_hold(lib):
-    # 272 MB of split partials needed; the library's fixed scratch is 16 MiB
-    assert lib.llama_attn_decode_noalloc(FAKE, FAKE, FAKE, FAKE, None, None, 64, 64, 8, 65536, 128,
+    # 35.7 MB of partials needed (1024 x 64 heads); the library's fixed scratch is 16 MiB
+    assert lib.llama_attn_decode_noalloc(FAKE, FAKE, FAKE, FAKE, None, None, 1024, 64, 8, 4096, 128,
                                          0.088, FAKE, 1, None) == 1
     # argument checks are the regular decode's
     assert lib.llama_attn_decode_noalloc(FAKE, FAKE, FAKE, None, None, None, 2, 8, 2, 100, 128,
