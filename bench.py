@@ -7,6 +7,10 @@ One JSON line on stdout (rank 0).  Two timed phases, each of exactly K steps
 after W warm-up steps, bracketed by a barrier and a device synchronisation on
 both sides, timed with CUDA events on the launching stream, max over ranks:
 
+Timed steps are CUDA-graph replays of one step's launches (captured through the
+public API; ``--no-graph`` launches them directly); the roofline figures come
+from a second pass with CUDA events around each library call.
+
 * prefill (headline ``value``): the 70B-shaped causal GQA workload
   (b1 S8192 H64 Hkv8 D128, RoPE theta 1e4 with linear factor 2.0, bf16).  One
   step = RoPE table from position ids + llama_attn_prefill (K rotation pass +
@@ -146,6 +150,30 @@ class ClockSampler:
         return out
 
 
+def _capture(step_fn):
+    """Capture one step (its kernel launches, through the public API) into a CUDA
+    graph; None if capture is not possible here (the steps then launch directly)."""
+    try:
+        return _capture_or_raise(step_fn)
+    except Exception as e:  # noqa: BLE001
+        print(f"bench: CUDA graph capture failed ({e}); launching directly", file=sys.stderr)
+        torch.cuda.synchronize()
+        return None
+
+
+def _capture_or_raise(step_fn):
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        step_fn()
+    torch.cuda.current_stream().wait_stream(side)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        step_fn()
+    torch.cuda.synchronize()
+    return graph
+
+
 # ----------------------------------------------------------------------------- our arm
 
 def run_ours(args, rank, ws, local):
@@ -201,18 +229,26 @@ def _prefill_phase(args, ws, local, dev, stream, line):
     for _ in range(args.warmup):
         prefill_step()
     torch.cuda.synchronize()
+    graph = None if args.no_graph else _capture(prefill_step)
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
            for _ in range(args.steps)]
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(local) as clk:
+        # whole steps (CUDA-graph replays of rope_table + llama_attn_prefill)
+        for _ in range(args.warmup):
+            graph.replay() if graph is not None else prefill_step()
         _barrier(ws)
         torch.cuda.synchronize()
         t0.record(stream)
         for i in range(args.steps):
-            prefill_step(evs[i])
+            graph.replay() if graph is not None else prefill_step()
         t1.record(stream)
         torch.cuda.synchronize()
         _barrier(ws)
+        # the prefill call alone, events around each call (roofline figure)
+        for i in range(args.steps):
+            prefill_step(evs[i])
+        torch.cuda.synchronize()
     clocks = clk.summary()
     ms_total = _max_over_ranks(t0.elapsed_time(t1), ws)
     ms_call = _max_over_ranks(statistics.mean(a.elapsed_time(b) for a, b in evs), ws)
@@ -271,6 +307,7 @@ def _prefill_phase(args, ws, local, dev, stream, line):
             "seq_len": cfg.seq,
             "parallelism": f"replicas x{ws}",
             "l2": "inputs larger than L2 (no flush)",
+            "launch": "cuda-graph replay" if graph is not None else "direct",
         },
         "roofline": {
             "bound": "tensor",
@@ -324,17 +361,25 @@ def _decode_phase(args, ws, local, dev, stream, line):
     for i in range(max(args.warmup, 3)):
         decode_step(i)
     torch.cuda.synchronize()
+    graphs = None if args.no_graph else [_capture(lambda i=i: decode_step(i)) for i in range(2)]
+    if graphs is not None and any(g_ is None for g_ in graphs):
+        graphs = None
     devs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
             for _ in range(dsteps)]
+    for i in range(max(args.warmup, 3)):
+        graphs[i % 2].replay() if graphs is not None else decode_step(i)
     _barrier(ws)
     torch.cuda.synchronize()
     d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     d0.record(stream)
     for i in range(dsteps):
-        decode_step(i, devs[i])
+        graphs[i % 2].replay() if graphs is not None else decode_step(i)
     d1.record(stream)
     torch.cuda.synchronize()
     _barrier(ws)
+    for i in range(dsteps):
+        decode_step(i, devs[i])
+    torch.cuda.synchronize()
     ms_dec_total = _max_over_ranks(d0.elapsed_time(d1), ws)
     ms_dec_call = _max_over_ranks(statistics.mean(a.elapsed_time(b) for a, b in devs), ws)
     dec_value = replicas.job_throughput(dbytes, dsteps, ms_dec_total, ws) / 1e9
@@ -342,6 +387,7 @@ def _decode_phase(args, ws, local, dev, stream, line):
     assert api.device_status() == api.LLAMA_OK
 
     line["decode"] = {
+        "launch": "cuda-graph replay" if graphs is not None else "direct",
         "value": round(dec_value, 1),
         "unit": "GB/s",
         "ms_per_step": round(ms_dec_total / dsteps, 4),
@@ -443,6 +489,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer e2e measurement")
+    ap.add_argument("--no-graph", action="store_true",
+                    help="launch every step directly instead of replaying a captured CUDA graph")
     ap.add_argument("--phase", choices=["all", "prefill", "decode"], default="all",
                     help="run only one timed phase (for profiling one kernel); the JSON "
                          "line then carries only that phase")

@@ -4,7 +4,7 @@
 // "GQA": several query heads share each K/V head, so one read of a K/V row
 // serves the whole group).
 //
-// Work is the flattened list of 256-row chunks of every sequence, where a
+// Work is the flattened list of 64-row chunks of every sequence, where a
 // sequence is (batch entry, K/V head, chunk of <= 8 query heads of its group),
 // built on the device from cache_lens.  A persistent grid (one CTA per SM)
 // gives each CTA an even share of the chunks -- no two shares differ by more
@@ -32,7 +32,7 @@
 namespace la {
 namespace dec {
 constexpr int TR = 64;           // cache rows per stage
-constexpr int CH = 256;          // rows per work chunk (granule of the even split)
+constexpr int CH = 64;           // rows per work chunk (granule of the even split)
 constexpr int NCW = 4;           // consumer warps (16 rows of a stage each)
 constexpr int NSTAGE = 5;        // ring depth
 constexpr int THREADS = (NCW + 1) * 32;
@@ -49,6 +49,7 @@ struct DecodeParams {
   const int* lens;         // [b]
   float* ws_home;          // [b, H, D + 4]: partial of the segment at a sequence's start
   float* ws_cta;           // [MAX_CTAS, 8, D + 4]: partial of a CTA's mid-sequence segment
+  int* ws_prefix;          // [b + 1]: chunks per sequence of batch entries < b (for the combine)
   int bsz, H, Hkv, L, group, hchunks;
   float scale_log2;        // scale * log2(e)
 };
@@ -142,21 +143,41 @@ __global__ void __launch_bounds__(dec::THREADS, 1) decode_bf16_kernel(
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int per_b = p.Hkv * p.hchunks;  // sequences per batch entry
 
-  // ---- chunk counts per batch entry, prefix-summed (identical in every CTA)
-  if (threadIdx.x == 0) {
-    int acc = 0;
-    for (int b = 0; b < p.bsz; ++b) {
+  // ---- chunk counts per batch entry, prefix-summed (identical in every CTA):
+  // each thread sums a contiguous run of entries, one thread scans the run
+  // totals, then each thread writes the prefixes of its run
+  {
+    __shared__ int run_total[THREADS];
+    const int per = (p.bsz + THREADS - 1) / THREADS;
+    const int lo = min(p.bsz, static_cast<int>(threadIdx.x) * per), hi = min(p.bsz, lo + per);
+    int sum = 0;
+    for (int b = lo; b < hi; ++b) sum += (clamp_len(p.lens[b], p.L) + CH - 1) / CH;
+    run_total[threadIdx.x] = sum;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      int acc = 0;
+      for (int i = 0; i < THREADS; ++i) {
+        const int v = run_total[i];
+        run_total[i] = acc;
+        acc += v;
+      }
+      s.chunk_prefix[p.bsz] = acc;
+      for (int i = 0; i < NSTAGE; ++i) {
+        mbar_init(&s.full[i], 1);
+        mbar_init(&s.empty[i], NCW);
+      }
+      fence_mbar_init();
+    }
+    __syncthreads();
+    int acc = run_total[threadIdx.x];
+    for (int b = lo; b < hi; ++b) {
       s.chunk_prefix[b] = acc;
       acc += (clamp_len(p.lens[b], p.L) + CH - 1) / CH;
     }
-    s.chunk_prefix[p.bsz] = acc;
-    for (int i = 0; i < NSTAGE; ++i) {
-      mbar_init(&s.full[i], 1);
-      mbar_init(&s.empty[i], NCW);
-    }
-    fence_mbar_init();
+    __syncthreads();
+    if (blockIdx.x == 0)
+      for (int b = threadIdx.x; b <= p.bsz; b += THREADS) p.ws_prefix[b] = s.chunk_prefix[b];
   }
-  __syncthreads();
   // the combine kernel may be scheduled now; it waits for this grid to finish
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const long long n_chunks = static_cast<long long>(s.chunk_prefix[p.bsz]) * per_b;
@@ -426,6 +447,7 @@ __global__ void __launch_bounds__(dec::THREADS, 1) decode_bf16_kernel(
 template <int D>
 __global__ void __launch_bounds__(D) decode_combine_kernel(const float* __restrict__ ws_home,
                                                            const float* __restrict__ ws_cta,
+                                                           const int* __restrict__ ws_prefix,
                                                            const int* __restrict__ lens,
                                                            __nv_bfloat16* __restrict__ out,
                                                            int bsz, int H, int Hkv, int L,
@@ -433,23 +455,14 @@ __global__ void __launch_bounds__(D) decode_combine_kernel(const float* __restri
   // the split kernel's writes are visible after this (programmatic dependent launch)
   asm volatile("griddepcontrol.wait;" ::: "memory");
   const int h = blockIdx.x, b = blockIdx.y, d = threadIdx.x;
-  __shared__ long long sh_prefix_b, sh_total;
-  if (d == 0) {
-    long long acc = 0, pre = 0;
-    for (int i = 0; i < bsz; ++i) {
-      if (i == b) pre = acc;
-      acc += (clamp_len(lens[i], L) + dec::CH - 1) / dec::CH;
-    }
-    sh_prefix_b = pre;
-    sh_total = acc;
-  }
-  __syncthreads();
+  const long long prefix_b = ws_prefix[b];
+  const long long total = ws_prefix[bsz];
   const int per_b = Hkv * hchunks;
   const int nch = (clamp_len(lens[b], L) + dec::CH - 1) / dec::CH;
   const int kvh = h / group, hq = h - kvh * group, hc = hq / 8, hh = hq % 8;
-  const long long n_chunks = sh_total * per_b;
+  const long long n_chunks = total * per_b;
   const long long G = n_ctas;
-  const long long P = sh_prefix_b * per_b + static_cast<long long>(kvh * hchunks + hc) * nch;
+  const long long P = prefix_b * per_b + static_cast<long long>(kvh * hchunks + hc) * nch;
   float mstar = -INFINITY, lsum = 0.f, acc = 0.f;
   auto add = [&](const float* part) {
     const float mc = part[D], lc = part[D + 1];

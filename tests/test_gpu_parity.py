@@ -190,6 +190,9 @@ DECODE_CASES = [
     (2, 16, 1, 128, 700, [0, 700]),          # MQA, an empty cache row
     (2, 32, 2, 64, 2000, [1024, 1999]),      # group 16: two head chunks
     (5, 12, 4, 128, 130, [63, 64, 65, 128, 129]),
+    (300, 8, 8, 64, 96, None),              # prefix runs of several batch entries per thread
+    (3, 8, 2, 128, 200, [0, 0, 0]),          # no work at all: zero output everywhere
+    (4, 16, 2, 128, 300, [-3, 301, 1000, 150]),  # lengths outside [0, L] are clamped
 ]
 
 
@@ -197,17 +200,22 @@ DECODE_CASES = [
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32], ids=["bf16", "fp32"])
 def test_decode_small(case, dtype):
     b, H, Hkv, D, L, lens = case
-    cfg, x = W.small_decode(b, H, Hkv, D, L, dtype, seed=sum(lens) + H,
-                            lens=torch.tensor(lens, dtype=torch.int32))
+    if lens is None:
+        lens = torch.randint(0, L + 1, (b,), generator=torch.Generator().manual_seed(b)).tolist()
+    clamped = [min(max(n, 0), L) for n in lens]
+    cfg, x = W.small_decode(b, H, Hkv, D, L, dtype, seed=sum(clamped) + H,
+                            lens=torch.tensor(clamped, dtype=torch.int32))
+    x["lens"] = torch.tensor(lens, dtype=torch.int32)  # the device sees the raw lengths
     dev = torch.device("cuda")
     cos, sin = api.rope_table(x["qpos"].view(-1, 1).to(dev), D, cfg.theta, cfg.factor)
     out = api.decode(x["q"].to(dev), x["k_cache"].to(dev), x["v_cache"].to(dev),
                      x["lens"].to(dev), cos.view(b, D), sin.view(b, D), scale=cfg.scale)
     torch.cuda.synchronize()
-    ref = oracle.decode(x["q"], x["k_cache"], x["v_cache"], x["lens"], x["qpos"],
+    ref = oracle.decode(x["q"], x["k_cache"], x["v_cache"], torch.tensor(clamped), x["qpos"],
                         theta=cfg.theta, factor=cfg.factor, scale=cfg.scale)
-    _check(out, ref, dtype, str(case))
-    for i, n in enumerate(lens):
+    if max(clamped) > 0:
+        _check(out, ref, dtype, str(case))
+    for i, n in enumerate(clamped):
         if n == 0:
             assert torch.all(out[i].float().cpu() == 0)
 
