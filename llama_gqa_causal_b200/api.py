@@ -16,6 +16,8 @@ from typing import Optional, Tuple
 
 import torch
 
+from . import build as _build
+
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libllama_attn.so")
 
@@ -50,13 +52,23 @@ class LlamaAttnError(RuntimeError):
 
 
 def load() -> ctypes.CDLL:
-    """Load the in-tree library (raises if it has not been built)."""
+    """Load the in-tree library.
+
+    Raises if it has not been built, or if it was built from sources other
+    than the ones now in the tree (a stale library would silently run old
+    kernels).
+    """
     global _lib
     if _lib is not None:
         return _lib
     if not os.path.exists(LIB_PATH):
         raise RuntimeError(
             f"{LIB_PATH} is missing: build it with `python -m llama_gqa_causal_b200.build`")
+    if os.path.abspath(LIB_PATH) == os.path.abspath(_build.LIB) and \
+            _build.built_hash() != _build.source_hash():
+        raise RuntimeError(
+            f"{LIB_PATH} was built from other sources than the ones in the tree: "
+            "rebuild it with `python -m llama_gqa_causal_b200.build`")
     lib = ctypes.CDLL(LIB_PATH)
     P, I, D, Z, F = ctypes.c_void_p, ctypes.c_int, ctypes.c_double, ctypes.c_size_t, ctypes.c_float
     lib.llama_rope_table.argtypes = [P, I, I, I, D, D, P, P, P]

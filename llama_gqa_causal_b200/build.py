@@ -11,6 +11,7 @@ from __future__ import annotations
 
 import argparse
 import glob
+import hashlib
 import os
 import subprocess
 import sys
@@ -20,6 +21,8 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libllama_attn.so")
+# Written beside the library by build(): the source hash it was compiled from.
+HASH_FILE = LIB + ".srchash"
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 
 FLAGS = [
@@ -35,11 +38,27 @@ def sources():
                   + glob.glob(os.path.join(INCLUDE, "*.h")))
 
 
+def source_hash() -> str:
+    """sha256 over every CUDA source and public header (names and contents)."""
+    h = hashlib.sha256()
+    for s in sources():
+        h.update(os.path.relpath(s, ROOT).encode())
+        with open(s, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def built_hash() -> str | None:
+    """Source hash recorded when the in-tree library was built (None if unknown)."""
+    try:
+        with open(HASH_FILE) as f:
+            return f.read().strip()
+    except OSError:
+        return None
+
+
 def needs_build() -> bool:
-    if not os.path.exists(LIB):
-        return True
-    t = os.path.getmtime(LIB)
-    return any(os.path.getmtime(s) > t for s in sources())
+    return not os.path.exists(LIB) or built_hash() != source_hash()
 
 
 def build(force: bool = False, verbose_ptxas: bool = False) -> str:
@@ -49,7 +68,12 @@ def build(force: bool = False, verbose_ptxas: bool = False) -> str:
            os.path.join(CSRC, "llama_attn.cu")]
     if verbose_ptxas:
         cmd.insert(1, "-Xptxas=-v")
+    digest = source_hash()
+    if os.path.exists(HASH_FILE):
+        os.remove(HASH_FILE)
     subprocess.check_call(cmd)
+    with open(HASH_FILE, "w") as f:
+        f.write(digest + "\n")
     return LIB
 
 

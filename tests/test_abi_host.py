@@ -153,3 +153,15 @@ def test_python_binding_refuses_cpu_tensors(lib):
 
 def test_build_flags_target_sm100a():
     assert "arch=compute_100a,code=sm_100a" in " ".join(build.FLAGS)
+
+
+def test_loader_refuses_a_library_built_from_other_sources(lib, monkeypatch):
+    # A library whose recorded source hash differs from the tree's sources
+    # would run old kernels under new tests; the loader must refuse it.
+    assert build.built_hash() == build.source_hash()
+    monkeypatch.setattr(api, "_lib", None)
+    monkeypatch.setattr(build, "built_hash", lambda: "0" * 64)
+    with pytest.raises(RuntimeError, match="other sources"):
+        api.load()
+    monkeypatch.undo()
+    assert api.load() is not None
