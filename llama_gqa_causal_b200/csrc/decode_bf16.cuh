@@ -49,7 +49,6 @@ struct DecodeParams {
   const int* lens;         // [b]
   float* ws_home;          // [b, H, D + 4]: partial of the segment at a sequence's start
   float* ws_cta;           // [MAX_CTAS, 8, D + 4]: partial of a CTA's mid-sequence segment
-  int* ws_prefix;          // [b + 1]: chunks per sequence of batch entries < b (for the combine)
   int bsz, H, Hkv, L, group, hchunks;
   float scale_log2;        // scale * log2(e)
 };
@@ -142,26 +141,29 @@ __global__ void __launch_bounds__(dec::THREADS, 1) decode_bf16_kernel(
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int per_b = p.Hkv * p.hchunks;  // sequences per batch entry
+  if (warp == NCW && elect_one()) {  // descriptor fetch overlaps the prologue
+    tma_prefetch_desc(&tm_k);
+    tma_prefetch_desc(&tm_v);
+  }
 
   // ---- chunk counts per batch entry, prefix-summed (identical in every CTA):
-  // each thread sums a contiguous run of entries, one thread scans the run
-  // totals, then each thread writes the prefixes of its run
+  // each thread sums a contiguous run of entries, the run totals are scanned
+  // with warp shuffles and the per-warp totals, then each thread writes the
+  // prefixes of its run
   {
-    __shared__ int run_total[THREADS];
+    __shared__ int warp_total[THREADS / 32];
     const int per = (p.bsz + THREADS - 1) / THREADS;
     const int lo = min(p.bsz, static_cast<int>(threadIdx.x) * per), hi = min(p.bsz, lo + per);
     int sum = 0;
     for (int b = lo; b < hi; ++b) sum += (clamp_len(p.lens[b], p.L) + CH - 1) / CH;
-    run_total[threadIdx.x] = sum;
-    __syncthreads();
+    int incl = sum;  // inclusive scan of the run totals within the warp
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    if (lane == 31) warp_total[warp] = incl;
     if (threadIdx.x == 0) {
-      int acc = 0;
-      for (int i = 0; i < THREADS; ++i) {
-        const int v = run_total[i];
-        run_total[i] = acc;
-        acc += v;
-      }
-      s.chunk_prefix[p.bsz] = acc;
       for (int i = 0; i < NSTAGE; ++i) {
         mbar_init(&s.full[i], 1);
         mbar_init(&s.empty[i], NCW);
@@ -169,14 +171,14 @@ __global__ void __launch_bounds__(dec::THREADS, 1) decode_bf16_kernel(
       fence_mbar_init();
     }
     __syncthreads();
-    int acc = run_total[threadIdx.x];
+    int acc = incl - sum;  // exclusive prefix of this thread's run
+    for (int w = 0; w < warp; ++w) acc += warp_total[w];
+    if (threadIdx.x == THREADS - 1) s.chunk_prefix[p.bsz] = acc + sum;
     for (int b = lo; b < hi; ++b) {
       s.chunk_prefix[b] = acc;
       acc += (clamp_len(p.lens[b], p.L) + CH - 1) / CH;
     }
     __syncthreads();
-    if (blockIdx.x == 0)
-      for (int b = threadIdx.x; b <= p.bsz; b += THREADS) p.ws_prefix[b] = s.chunk_prefix[b];
   }
   // the combine kernel may be scheduled now; it waits for this grid to finish
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -186,11 +188,6 @@ __global__ void __launch_bounds__(dec::THREADS, 1) decode_bf16_kernel(
   if (x0 >= x1) return;  // uniform across the CTA: no share
 
   if (warp == NCW) {  // ---------------------------------------------- TMA producer
-    if (elect_one()) {
-      tma_prefetch_desc(&tm_k);
-      tma_prefetch_desc(&tm_v);
-    }
-    __syncwarp();
     int b = 0;
     int it = 0;  // tiles issued
     bool ok = true;
@@ -440,55 +437,131 @@ __global__ void __launch_bounds__(dec::THREADS, 1) decode_bf16_kernel(
   }
 }
 
-// Merge the partials of one (b, head).  Its sequence's segments start at the
-// sequence's first chunk (home slot) and at every chunk where some CTA's share
-// begins inside the sequence (that CTA's own slot).
+// Merge the partials of the heads of one sequence (batch entry, K/V head,
+// chunk of <= 8 query heads): one warp per head, each lane D/32 dimensions.
+// The sequence's segments start at its first chunk (home slot) and at every
+// chunk where some CTA's share begins inside it (that CTA's own slot).
 //   m* = max_s m_s,  l = sum_s l_s 2^(m_s - m*),  o = sum_s o_s 2^(m_s - m*) / l.
+// Everything that depends only on cache_lens (the chunk prefix of the batch
+// entry, the segment starts) is computed before the wait for the split kernel,
+// and the partials of up to kEager segments are then loaded at once.
+namespace dec {
+constexpr int COMBINE_THREADS = 256;  // 8 warps = the heads of one sequence
+}
 template <int D>
-__global__ void __launch_bounds__(D) decode_combine_kernel(const float* __restrict__ ws_home,
-                                                           const float* __restrict__ ws_cta,
-                                                           const int* __restrict__ ws_prefix,
-                                                           const int* __restrict__ lens,
-                                                           __nv_bfloat16* __restrict__ out,
-                                                           int bsz, int H, int Hkv, int L,
-                                                           int group, int hchunks, int n_ctas) {
-  // the split kernel's writes are visible after this (programmatic dependent launch)
-  asm volatile("griddepcontrol.wait;" ::: "memory");
-  const int h = blockIdx.x, b = blockIdx.y, d = threadIdx.x;
-  const long long prefix_b = ws_prefix[b];
-  const long long total = ws_prefix[bsz];
+__global__ void __launch_bounds__(dec::COMBINE_THREADS) decode_combine_kernel(
+    const float* __restrict__ ws_home, const float* __restrict__ ws_cta,
+    const int* __restrict__ lens, __nv_bfloat16* __restrict__ out, int bsz, int H, int Hkv, int L,
+    int group, int hchunks, int n_ctas) {
+  constexpr int kEager = 4;
+  constexpr int VEC = D / 32;  // dimensions per lane
+  constexpr int NW = dec::COMBINE_THREADS / 32;
+  const int seq = blockIdx.x, b = blockIdx.y;
+  const int kvh = seq / hchunks, hc = seq - kvh * hchunks;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  // chunks of batch entries < b and of all entries: block-wide sums over lens
+  __shared__ long long red[2][NW];
+  long long before = 0, all = 0;
+  for (int e = threadIdx.x; e < bsz; e += dec::COMBINE_THREADS) {
+    const int c = (clamp_len(lens[e], L) + dec::CH - 1) / dec::CH;
+    all += c;
+    if (e < b) before += c;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    before += __shfl_xor_sync(0xffffffffu, before, o);
+    all += __shfl_xor_sync(0xffffffffu, all, o);
+  }
+  if (lane == 0) {
+    red[0][warp] = before;
+    red[1][warp] = all;
+  }
+  __syncthreads();
+  long long prefix_b = 0, total = 0;
+#pragma unroll
+  for (int w = 0; w < NW; ++w) {
+    prefix_b += red[0][w];
+    total += red[1][w];
+  }
   const int per_b = Hkv * hchunks;
   const int nch = (clamp_len(lens[b], L) + dec::CH - 1) / dec::CH;
-  const int kvh = h / group, hq = h - kvh * group, hc = hq / 8, hh = hq % 8;
   const long long n_chunks = total * per_b;
   const long long G = n_ctas;
-  const long long P = prefix_b * per_b + static_cast<long long>(kvh * hchunks + hc) * nch;
-  float mstar = -INFINITY, lsum = 0.f, acc = 0.f;
-  auto add = [&](const float* part) {
-    const float mc = part[D], lc = part[D + 1];
-    const float m_new = fmaxf(mstar, mc);
-    const float fo = (mstar == -INFINITY) ? 0.f : ex2_approx(mstar - m_new);
-    const float fc = ex2_approx(mc - m_new);
-    lsum = lsum * fo + lc * fc;
-    acc = acc * fo + part[d] * fc;
-    mstar = m_new;
-  };
-  if (nch > 0) {
-    add(ws_home + (static_cast<size_t>(b) * H + h) * dec::part_stride(D));
-    // CTA shares that begin strictly inside [P, P + nch); equal starts mean empty
-    // shares, and the owner of a start is the last CTA with that start
-    long long last_start = P;
-    for (long long gi = share_owner(P, n_chunks, G) + 1; gi < G; ++gi) {
+  const long long P = prefix_b * per_b + static_cast<long long>(seq) * nch;
+  // owners of the CTA shares that begin strictly inside [P, P + nch); equal
+  // starts mean empty shares, and the owner of a start is the last CTA with it
+  long long gi = (nch > 0) ? share_owner(P, n_chunks, G) + 1 : G;
+  long long last_start = P;
+  auto next_owner = [&]() -> long long {
+    for (; gi < G; ++gi) {
       const long long st = share_start(gi, n_chunks, G);
       if (st >= P + nch) break;
       if (st == last_start) continue;
       last_start = st;
-      const long long owner = share_owner(st, n_chunks, G);
-      add(ws_cta + (static_cast<size_t>(owner) * 8 + hh) * dec::part_stride(D));
+      ++gi;
+      return share_owner(st, n_chunks, G);
+    }
+    gi = G;
+    return -1;
+  };
+  long long own[kEager];
+#pragma unroll
+  for (int k = 0; k < kEager; ++k) own[k] = next_owner();
+
+  const int hq = hc * 8 + warp;  // query head within the group
+  const bool active = hq < group;
+  const int head = kvh * group + hq;
+  // the split kernel's writes are visible after this (programmatic dependent launch)
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  if (!active) return;
+  float mstar = -INFINITY, lsum = 0.f, acc[VEC];
+#pragma unroll
+  for (int v = 0; v < VEC; ++v) acc[v] = 0.f;
+  auto add = [&](float mc, float lc, const float (&oc)[VEC]) {
+    const float m_new = fmaxf(mstar, mc);
+    const float fo = (mstar == -INFINITY) ? 0.f : ex2_approx(mstar - m_new);
+    const float fc = ex2_approx(mc - m_new);
+    lsum = lsum * fo + lc * fc;
+#pragma unroll
+    for (int v = 0; v < VEC; ++v) acc[v] = acc[v] * fo + oc[v] * fc;
+    mstar = m_new;
+  };
+  auto load = [&](const float* part, float& m, float& l, float (&o)[VEC]) {
+    m = part[D];
+    l = part[D + 1];
+#pragma unroll
+    for (int v = 0; v < VEC; v += 2) {
+      const float2 x = *reinterpret_cast<const float2*>(part + lane * VEC + v);
+      o[v] = x.x;
+      o[v + 1] = x.y;
+    }
+  };
+  if (nch > 0) {
+    float pm[kEager + 1], pl[kEager + 1], po[kEager + 1][VEC];
+    load(ws_home + (static_cast<size_t>(b) * H + head) * dec::part_stride(D), pm[0], pl[0], po[0]);
+#pragma unroll
+    for (int k = 0; k < kEager; ++k)
+      if (own[k] >= 0)
+        load(ws_cta + (static_cast<size_t>(own[k]) * 8 + warp) * dec::part_stride(D), pm[k + 1],
+             pl[k + 1], po[k + 1]);
+    add(pm[0], pl[0], po[0]);
+#pragma unroll
+    for (int k = 0; k < kEager; ++k)
+      if (own[k] >= 0) add(pm[k + 1], pl[k + 1], po[k + 1]);
+    // sequences split over more CTAs than that (short batches): the rest one by one
+    if (own[kEager - 1] >= 0) {
+      for (long long ow = next_owner(); ow >= 0; ow = next_owner()) {
+        float m, l, o[VEC];
+        load(ws_cta + (static_cast<size_t>(ow) * 8 + warp) * dec::part_stride(D), m, l, o);
+        add(m, l, o);
+      }
     }
   }
-  const float r = (lsum > 0.f) ? acc / lsum : 0.f;
-  out[(static_cast<size_t>(b) * H + h) * D + d] = __float2bfloat16_rn(r);
+  const float inv = (lsum > 0.f) ? 1.f / lsum : 0.f;
+  __nv_bfloat16* dst = out + (static_cast<size_t>(b) * H + head) * D + lane * VEC;
+#pragma unroll
+  for (int v = 0; v < VEC; v += 2)
+    *reinterpret_cast<uint32_t*>(dst + v) = pack_bf16x2(acc[v] * inv, acc[v + 1] * inv);
 }
 
 }  // namespace la

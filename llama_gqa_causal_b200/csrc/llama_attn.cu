@@ -199,8 +199,6 @@ int decode_bf16(const void* q, const void* kc, const void* vc, const int* lens, 
   p.lens = lens;
   p.ws_home = static_cast<float*>(workspace);
   p.ws_cta = p.ws_home + static_cast<size_t>(bsz) * H * la::dec::part_stride(D);
-  p.ws_prefix = reinterpret_cast<int*>(p.ws_cta + static_cast<size_t>(la::dec::MAX_CTAS) * 8 *
-                                                      la::dec::part_stride(D));
   p.bsz = bsz;
   p.H = H;
   p.Hkv = Hkv;
@@ -215,8 +213,8 @@ int decode_bf16(const void* q, const void* kc, const void* vc, const int* lens, 
   // the combine launches as a programmatic dependent of the split kernel: its
   // blocks are scheduled while the split kernel drains and wait on the device
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(H, bsz);
-  cfg.blockDim = dim3(D);
+  cfg.gridDim = dim3(Hkv * p.hchunks, bsz);
+  cfg.blockDim = dim3(la::dec::COMBINE_THREADS);
   cfg.dynamicSmemBytes = 0;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
@@ -226,10 +224,9 @@ int decode_bf16(const void* q, const void* kc, const void* vc, const int* lens, 
   cfg.numAttrs = 1;
   const float* home = p.ws_home;
   const float* ctas = p.ws_cta;
-  const int* prefix = p.ws_prefix;
   __nv_bfloat16* o = static_cast<__nv_bfloat16*>(out);
   int group = p.group, hchunks = p.hchunks;
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, la::decode_combine_kernel<D>, home, ctas, prefix,
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, la::decode_combine_kernel<D>, home, ctas,
                                            lens, o, bsz, H, Hkv, L, group, hchunks, n_ctas);
   if (e != cudaSuccess) {
     fprintf(stderr, "llama_attn: combine launch failed: %s\n", cudaGetErrorString(e));
@@ -342,11 +339,9 @@ int llama_attn_prefill(const void* q, const void* k, const void* v, const float*
 
 size_t llama_attn_decode_workspace_bytes(int bsz, int n_heads, int max_cache_len, int head_dim) {
   if (bsz < 1 || n_heads < 1 || max_cache_len < 1 || head_dim < 1) return 0;
-  // one partial per (batch, head) plus one per (CTA, head of an 8-head chunk),
-  // then the per-batch chunk prefix (bsz + 1 ints, rounded up to 16 bytes)
+  // one partial per (batch, head) plus one per (CTA, head of an 8-head chunk)
   const size_t rows = static_cast<size_t>(bsz) * n_heads + static_cast<size_t>(la::dec::MAX_CTAS) * 8;
-  return rows * la::dec::part_stride(head_dim) * sizeof(float) +
-         ((static_cast<size_t>(bsz) + 1) * sizeof(int) + 15) / 16 * 16;
+  return rows * la::dec::part_stride(head_dim) * sizeof(float);
 }
 
 int llama_attn_decode(const void* q, const void* k_cache, const void* v_cache,

@@ -56,10 +56,10 @@ def test_workspace_sizes(lib):
     assert lib.llama_attn_prefill_workspace_bytes(1, 64, 8, 8192, 128, 1, 0) == 0
     assert lib.llama_attn_prefill_workspace_bytes(1, 4, 2, 64, 64, 0, 1) == 0
     # decode: one partial row of D + 4 floats per (b, head) and per (CTA, head of
-    # an 8-head chunk) for up to 256 CTAs, then the per-batch chunk prefix
-    assert lib.llama_attn_decode_workspace_bytes(32, 64, 4096, 128) == (32 * 64 + 256 * 8) * 132 * 4 + 144
-    assert lib.llama_attn_decode_workspace_bytes(2, 4, 513, 64) == (2 * 4 + 256 * 8) * 68 * 4 + 16
-    assert lib.llama_attn_decode_workspace_bytes(2, 4, 1 << 20, 64) == (2 * 4 + 256 * 8) * 68 * 4 + 16
+    # an 8-head chunk) for up to 256 CTAs; independent of the cache length
+    assert lib.llama_attn_decode_workspace_bytes(32, 64, 4096, 128) == (32 * 64 + 256 * 8) * 132 * 4
+    assert lib.llama_attn_decode_workspace_bytes(2, 4, 513, 64) == (2 * 4 + 256 * 8) * 68 * 4
+    assert lib.llama_attn_decode_workspace_bytes(2, 4, 1 << 20, 64) == (2 * 4 + 256 * 8) * 68 * 4
     assert lib.llama_attn_decode_workspace_bytes(0, 4, 513, 64) == 0
 
 
