@@ -21,6 +21,11 @@ from a second pass with CUDA events around each library call.
   llama_attn_decode (split-KV kernel + combine).  Bytes = K and V rows read,
   2 * sum(len_b) * Hkv * D * 2.
 
+``--phase configs`` instead times every named workload (the five shapes the
+parity tests cover) through the public API, one JSON line per workload, with
+CUDA events around each call (direct launches); it is a report, not the
+benchmark line.
+
 Inputs are larger than L2 (126 MB) in both phases (prefill: q 134 MB, out
 134 MB; decode: two alternating 537 MB caches, ~302 MB read per step), so no
 L2 flush is needed between steps.  Multi-GPU runs are independent replicas
@@ -481,6 +486,67 @@ def run_reference(args, rank, ws):
     }
 
 
+def run_configs(args):
+    """One JSON line per named workload: mean duration of the library call."""
+    from llama_gqa_causal_b200 import api
+    api.load()
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream()
+    peak_burst, _, hbm, peak_src = _peaks()
+    steps = max(args.steps, 10)
+
+    def timed(call):
+        for _ in range(args.warmup):
+            call()
+        torch.cuda.synchronize()
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(steps)]
+        for a, b in evs:
+            a.record(stream)
+            call()
+            b.record(stream)
+        torch.cuda.synchronize()
+        assert api.device_status() == api.LLAMA_OK
+        return statistics.mean(a.elapsed_time(b) for a, b in evs)
+
+    for cfg in W.PREFILL_CONFIGS.values():
+        x = W.prefill_inputs(cfg)
+        q, k, v = (x[n].to(dev) for n in ("q", "k", "v"))
+        cos = sin = None
+        if x["pos"] is not None:
+            cos, sin = api.rope_table(x["pos"].to(dev), cfg.head_dim, cfg.theta, cfg.factor)
+        out = torch.empty(cfg.bsz, cfg.seq, cfg.n_heads * cfg.head_dim, device=dev, dtype=cfg.dtype)
+        wsp = torch.empty(max(1, api.prefill_workspace_bytes(cfg.bsz, cfg.n_heads, cfg.n_kv_heads,
+                                                             cfg.seq, cfg.head_dim, cfg.dtype,
+                                                             cos is not None)),
+                          device=dev, dtype=torch.uint8)
+        ms = timed(lambda: api.prefill(q, k, v, cos, sin, causal=cfg.causal, scale=cfg.scale,
+                                       out=out, workspace=wsp))
+        tflops = cfg.flops() / (ms * 1e-3) / 1e12
+        print(json.dumps({"phase": "configs", "workload": cfg.name, "dtype": str(cfg.dtype).split(".")[-1],
+                          "ms_per_call": round(ms, 5), "value": round(tflops, 2), "unit": "TFLOP/s",
+                          "frac": round(tflops / peak_burst, 4),
+                          "peak": f"{peak_burst} TFLOP/s ({peak_src} bf16 burst)"}), flush=True)
+        del q, k, v, out, wsp, x
+    for cfg in W.DECODE_CONFIGS.values():
+        x = W.decode_inputs(cfg)
+        d = {n: x[n].to(dev) for n in ("q", "k_cache", "v_cache", "lens", "qpos")}
+        cos, sin = api.rope_table(d["qpos"].view(-1, 1), cfg.head_dim, cfg.theta, cfg.factor)
+        cos, sin = cos.view(cfg.bsz, -1), sin.view(cfg.bsz, -1)
+        out = torch.empty(cfg.bsz, cfg.n_heads * cfg.head_dim, device=dev, dtype=cfg.dtype)
+        wsp = torch.empty(api.decode_workspace_bytes(cfg.bsz, cfg.n_heads, cfg.max_cache_len,
+                                                     cfg.head_dim), device=dev, dtype=torch.uint8)
+        ms = timed(lambda: api.decode(d["q"], d["k_cache"], d["v_cache"], d["lens"], cos, sin,
+                                      scale=cfg.scale, out=out, workspace=wsp))
+        nbytes = int(2 * x["lens"].to(torch.int64).sum().item() * cfg.n_kv_heads * cfg.head_dim * 2)
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        print(json.dumps({"phase": "configs", "workload": cfg.name, "dtype": str(cfg.dtype).split(".")[-1],
+                          "ms_per_call": round(ms, 5), "value": round(gbs, 1), "unit": "GB/s",
+                          "frac": round(gbs / hbm, 4), "peak": f"{hbm} GB/s ({peak_src} copy)"}),
+              flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -491,12 +557,17 @@ def main():
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer e2e measurement")
     ap.add_argument("--no-graph", action="store_true",
                     help="launch every step directly instead of replaying a captured CUDA graph")
-    ap.add_argument("--phase", choices=["all", "prefill", "decode"], default="all",
-                    help="run only one timed phase (for profiling one kernel); the JSON "
-                         "line then carries only that phase")
+    ap.add_argument("--phase", choices=["all", "prefill", "decode", "configs"], default="all",
+                    help="run only one timed phase (for profiling one kernel; the JSON line "
+                         "then carries only that phase), or 'configs': one line per named "
+                         "workload, single GPU")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
+    if args.phase == "configs":
+        if int(os.environ.get("RANK", "0")) == 0:
+            run_configs(args)
+        return
     if args.impl == "reference":
         rank = int(os.environ.get("RANK", "0"))
         line = run_reference(args, rank, int(os.environ.get("WORLD_SIZE", "1")))

@@ -118,7 +118,8 @@ size_t llama_attn_decode_workspace_bytes(int bsz, int n_heads, int max_cache_len
  *   workspace  caller-owned device scratch of at least
  *              llama_attn_decode_workspace_bytes(...) bytes
  * Errors: as llama_attn_prefill, plus INVALID_ARG for max_cache_len < 1 or a
- * NULL cache_lens.
+ * NULL cache_lens, and UNSUPPORTED for bf16 with bsz > 4096 (the bf16 kernel
+ * keeps a per-batch prefix of chunk counts in shared memory).
  */
 int llama_attn_decode(const void* q, const void* k_cache, const void* v_cache,
                       const int* cache_lens, const float* cos, const float* sin, int bsz,

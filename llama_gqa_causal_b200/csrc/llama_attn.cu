@@ -179,6 +179,9 @@ int sm_count() {
   return count[dev];
 }
 
+static_assert(sizeof(la::DecSmem<128>) + 1024 <= 227 * 1024, "decode shared memory exceeds 227 KB");
+static_assert(sizeof(la::PfSmem<128>) + 1024 <= 227 * 1024, "prefill shared memory exceeds 227 KB");
+
 template <int D>
 int decode_bf16(const void* q, const void* kc, const void* vc, const int* lens, const float* cos,
                 const float* sin, int bsz, int H, int Hkv, int L, float scale, void* out,

@@ -28,3 +28,16 @@ def pytest_collection_modifyitems(config, items):
     for item in items:
         if "gpu" in item.keywords:
             item.add_marker(skip)
+
+
+# (workload, dtype, max abs error, mean abs error) of the named-workload parity
+# checks, printed after the run so a log carries the achieved accuracy
+PARITY_REPORT = []
+
+
+def pytest_terminal_summary(terminalreporter, exitstatus, config):
+    if not PARITY_REPORT:
+        return
+    terminalreporter.write_sep("-", "parity against the fp64 oracle (named workloads)")
+    for name, dtype, mx, mean in PARITY_REPORT:
+        terminalreporter.write_line(f"{name:12s} {dtype:9s} max abs {mx:.3e}  mean abs {mean:.3e}")

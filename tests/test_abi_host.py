@@ -118,6 +118,7 @@ def _decode(lib, **kw):
     (dict(vc=FAKE + 4), 1),
     (dict(dtype=-1), 1),
     (dict(D=80), 2),
+    (dict(bsz=4097), 2),
 ])
 def test_decode_rejects(lib, kw, status):
     assert _decode(lib, **kw) == status

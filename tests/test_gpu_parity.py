@@ -16,6 +16,7 @@ import pytest
 import torch
 
 import oracle
+from conftest import PARITY_REPORT
 from llama_gqa_causal_b200 import api, workloads as W
 
 pytestmark = pytest.mark.gpu
@@ -25,7 +26,7 @@ BF16_MAX = 2e-2
 BF16_MEAN = 2e-3
 
 
-def _check(gpu, ref, dtype, what=""):
+def _check(gpu, ref, dtype, what="", report=False):
     g = gpu.detach().float().cpu().double().numpy()
     sel = ~np.isnan(ref)
     assert sel.any()
@@ -36,6 +37,8 @@ def _check(gpu, ref, dtype, what=""):
     else:
         assert err.max() <= BF16_MAX, f"{what}: max abs {err.max():.3e}"
         assert err.mean() <= BF16_MEAN, f"{what}: mean abs {err.mean():.3e}"
+    if report:
+        PARITY_REPORT.append((what, str(dtype).split(".")[-1], float(err.max()), float(err.mean())))
     return err.max(), err.mean()
 
 
@@ -77,7 +80,7 @@ def test_tiny_fp32_workload():
     cfg = W.TINY_FP32
     x = W.prefill_inputs(cfg)
     out = _gpu_prefill(cfg, x)
-    _check(out, _oracle_prefill(cfg, x), torch.float32, cfg.name)
+    _check(out, _oracle_prefill(cfg, x), torch.float32, cfg.name, report=True)
 
 
 def test_mha_bf16_workload_shape_and_values():
@@ -85,7 +88,7 @@ def test_mha_bf16_workload_shape_and_values():
     x = W.prefill_inputs(cfg)
     out = _gpu_prefill(cfg, x)
     assert tuple(out.shape) == (4, 128, 4096)  # the tensor-parallel demo's full output shape
-    _check(out, _oracle_prefill(cfg, x), torch.bfloat16, cfg.name)
+    _check(out, _oracle_prefill(cfg, x), torch.bfloat16, cfg.name, report=True)
 
 
 def _windows(S):
@@ -102,7 +105,7 @@ def test_full_size_prefill_workloads_sampled(name):
     for lo, hi in _windows(cfg.seq):
         part = _oracle_prefill(cfg, x, rows=(lo, hi))
         ref[:, lo:hi] = part[:, lo:hi]
-    _check(out, ref, torch.bfloat16, name)
+    _check(out, ref, torch.bfloat16, name + " (sampled rows)", report=True)
 
 
 def test_decode70b_workload():
@@ -116,7 +119,7 @@ def test_decode70b_workload():
     torch.cuda.synchronize()
     ref = oracle.decode(x["q"], x["k_cache"], x["v_cache"], x["lens"], x["qpos"],
                         theta=cfg.theta, factor=cfg.factor, scale=cfg.scale)
-    _check(out, ref, torch.bfloat16, cfg.name)
+    _check(out, ref, torch.bfloat16, cfg.name, report=True)
     assert api.device_status() == api.LLAMA_OK
 
 
