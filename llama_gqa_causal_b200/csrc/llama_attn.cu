@@ -111,7 +111,7 @@ int prefill_bf16(const void* q, const void* k, const void* v, const float* cos, 
     if (int e = launch_status()) return e;
     k_src = workspace;
   }
-  CUtensorMap tq, tk, tv;
+  CUtensorMap tq, tk, tv, to;
   const cuuint64_t qdims[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(H),
                                static_cast<cuuint64_t>(S), static_cast<cuuint64_t>(bsz)};
   const cuuint64_t qstrides[3] = {static_cast<cuuint64_t>(D) * 2,
@@ -119,6 +119,9 @@ int prefill_bf16(const void* q, const void* k, const void* v, const float* cos, 
                                   static_cast<cuuint64_t>(S) * H * D * 2};
   const cuuint32_t qbox[4] = {64, 1, static_cast<cuuint32_t>(la::pf::BM), 1};
   if (!make_map(&tq, q, 4, qdims, qstrides, qbox)) return LLAMA_ERR_CUDA;
+  // out [b, S, H*D] has q's layout; each warp stores 32 rows
+  const cuuint32_t obox[4] = {64, 1, 32, 1};
+  if (!make_map(&to, out, 4, qdims, qstrides, obox)) return LLAMA_ERR_CUDA;
   const cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(Hkv),
                               static_cast<cuuint64_t>(S), static_cast<cuuint64_t>(bsz)};
   const cuuint64_t strides[3] = {static_cast<cuuint64_t>(D) * 2,
@@ -148,7 +151,7 @@ int prefill_bf16(const void* q, const void* k, const void* v, const float* cos, 
   if (!ensure_smem_attr<la::prefill_sm100_kernel<D>>(smem)) return LLAMA_ERR_CUDA;
   const long long grid = static_cast<long long>(bsz) * Hkv * p.ctas_per_kvh;
   if (grid > 0x7fffffffLL) return LLAMA_ERR_INVALID_ARG;
-  la::prefill_sm100_kernel<D><<<static_cast<unsigned>(grid), la::pf::THREADS, smem, st>>>(tq, tk, tv, p);
+  la::prefill_sm100_kernel<D><<<static_cast<unsigned>(grid), la::pf::THREADS, smem, st>>>(tq, tk, tv, to, p);
   return launch_status();
 }
 

@@ -96,7 +96,8 @@ template <int D>
 __global__ void __launch_bounds__(pf::THREADS, 1)
     prefill_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                          const __grid_constant__ CUtensorMap tm_k,
-                         const __grid_constant__ CUtensorMap tm_v, PrefillParams p) {
+                         const __grid_constant__ CUtensorMap tm_v,
+                         const __grid_constant__ CUtensorMap tm_out, PrefillParams p) {
   using namespace pf;
   constexpr int CB = D / 64;                       // 64-column swizzle blocks per row
   constexpr uint32_t BLOCK_BYTES = BM * 128;       // one [128 rows x 64 cols] bf16 block
@@ -165,6 +166,7 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
+      tma_prefetch_desc(&tm_out);
       // the two Q tiles (raw; rotated in shared memory by their softmax warps)
       mbar_arrive_expect_tx(&s.q_loaded[0], TILE_BYTES);
 #pragma unroll
@@ -330,7 +332,6 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
     if (n_kv > 0) {
       const int head = t ? head1 : head0;
       const int i = my_pb * BM + r;  // query position (sequence index)
-      const bool row_valid = i < p.S;
       // ---- stage Q: the raw tile arrives by TMA; rotate it in shared memory.
       // Warp-cooperative: per step a warp takes 32 / (D/4) rows, each lane one
       // bf16 pair (d, d+1) of the first half and its partner pair d + D/2, with
@@ -507,29 +508,44 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
         if (edge) tile(std::true_type{});
         else tile(std::false_type{});
       }
-      // ---- epilogue: O / l -> bf16 -> out[b, i, head*D : head*D + D]
+      // ---- epilogue: O / l -> bf16 -> out[b, i, head*D : head*D + D].  Each warp
+      // writes its 32 rows into the unit's Q tile buffer (free: every MMA has
+      // completed once O is final) in the same 128-byte swizzle, then one lane
+      // stores them with TMA (rows past S are clipped by the tensor map) and
+      // waits until the copy has read shared memory.
       if (ok && mbar_wait(&s.o_full[t], 0)) {
         tc_fence_after();
         const float inv = (l_sum > 0.f) ? 1.f / l_sum : 0.f;
-        __nv_bfloat16* orow = p.out + (static_cast<size_t>(b) * p.S + i) * (static_cast<size_t>(p.H) * D) +
-                              static_cast<size_t>(head) * D;
+        uint8_t* ob = reinterpret_cast<uint8_t*>(&s.q[t][0]);
+        const uint32_t row = static_cast<uint32_t>(r) * 128;
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
           uint32_t orr[32];
           tmem_ld32(my_o + lane_off + c * 32, orr);
           tmem_ld_wait(orr);
-          if (row_valid) {
+          const int cb = (c * 32) / 64;
 #pragma unroll
-            for (int e = 0; e < 32; e += 8) {
-              uint4 w;
-              w.x = pack_bf16x2(__uint_as_float(orr[e]) * inv, __uint_as_float(orr[e + 1]) * inv);
-              w.y = pack_bf16x2(__uint_as_float(orr[e + 2]) * inv, __uint_as_float(orr[e + 3]) * inv);
-              w.z = pack_bf16x2(__uint_as_float(orr[e + 4]) * inv, __uint_as_float(orr[e + 5]) * inv);
-              w.w = pack_bf16x2(__uint_as_float(orr[e + 6]) * inv, __uint_as_float(orr[e + 7]) * inv);
-              *reinterpret_cast<uint4*>(orow + c * 32 + e) = w;
-            }
+          for (int e = 0; e < 32; e += 8) {
+            uint4 w;
+            w.x = pack_bf16x2(__uint_as_float(orr[e]) * inv, __uint_as_float(orr[e + 1]) * inv);
+            w.y = pack_bf16x2(__uint_as_float(orr[e + 2]) * inv, __uint_as_float(orr[e + 3]) * inv);
+            w.z = pack_bf16x2(__uint_as_float(orr[e + 4]) * inv, __uint_as_float(orr[e + 5]) * inv);
+            w.w = pack_bf16x2(__uint_as_float(orr[e + 6]) * inv, __uint_as_float(orr[e + 7]) * inv);
+            const uint32_t chunk = static_cast<uint32_t>(((c * 32) % 64 + e) / 8);
+            *reinterpret_cast<uint4*>(ob + cb * BLOCK_BYTES + row + ((chunk ^ (r & 7)) << 4)) = w;
           }
         }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0 && my_pb * BM + quarter * 32 < p.S) {  // the box holds a row below S
+#pragma unroll
+          for (int cb = 0; cb < CB; ++cb)
+            tma_store_4d(&tm_out, ob + cb * BLOCK_BYTES + quarter * 32 * 128, cb * 64, head,
+                         my_pb * BM + quarter * 32, b);
+          bulk_commit_group();
+          bulk_wait_group_read0();
+        }
+        __syncwarp();
       }
     }
   }
