@@ -525,7 +525,7 @@ def run_configs(args):
     torch.cuda.set_device(dev)
     stream = torch.cuda.current_stream()
     peak_burst, _, hbm, peak_src = _peaks()
-    steps = max(args.steps, 10)
+    steps = max(args.steps, 1)
 
     def timed(call):
         for _ in range(args.warmup):
@@ -541,7 +541,12 @@ def run_configs(args):
         assert api.device_status() == api.LLAMA_OK
         return statistics.mean(a.elapsed_time(b) for a, b in evs)
 
+    def wanted(cfg):
+        return args.workload in (None, cfg.name)
+
     for cfg in W.PREFILL_CONFIGS.values():
+        if not wanted(cfg):
+            continue
         x = W.prefill_inputs(cfg)
         q, k, v = (x[n].to(dev) for n in ("q", "k", "v"))
         cos = sin = None
@@ -561,6 +566,8 @@ def run_configs(args):
                           "peak": f"{peak_burst} TFLOP/s ({peak_src} bf16 burst)"}), flush=True)
         del q, k, v, out, wsp, x
     for cfg in W.DECODE_CONFIGS.values():
+        if not wanted(cfg):
+            continue
         x = W.decode_inputs(cfg)
         d = {n: x[n].to(dev) for n in ("q", "k_cache", "v_cache", "lens", "qpos")}
         cos, sin = api.rope_table(d["qpos"].view(-1, 1), cfg.head_dim, cfg.theta, cfg.factor)
@@ -592,6 +599,9 @@ def main():
                     help="run only one timed phase (for profiling one kernel; the JSON line "
                          "then carries only that phase), or 'configs': one line per named "
                          "workload, single GPU")
+    ap.add_argument("--workload", default=None,
+                    choices=sorted(list(W.PREFILL_CONFIGS) + list(W.DECODE_CONFIGS)),
+                    help="with --phase configs: time only this named workload")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

@@ -145,6 +145,13 @@ int prefill_bf16(const void* q, const void* k, const void* v, const float* cos, 
   p.n_pb = (S + la::pf::BM - 1) / la::pf::BM;
   p.n_kb = (S + la::pf::BN - 1) / la::pf::BN;
   p.ctas_per_kvh = (p.group * p.n_pb + la::pf::NQ - 1) / la::pf::NQ;
+  {
+    // bundles of (batch, K/V head) pairs whose K' and V take at most 48 MB,
+    // well inside the 126 MB L2 beside the streamed q and out tiles
+    const size_t kv_bytes = static_cast<size_t>(S) * D * 2 * 2;
+    const size_t per = std::max<size_t>(1, (size_t{48} << 20) / kv_bytes);
+    p.bkv_per_bundle = static_cast<int>(std::min<size_t>(per, static_cast<size_t>(bsz) * Hkv));
+  }
   p.causal = causal ? 1 : 0;
   p.scale_log2 = scale * 1.4426950408889634f;
   const size_t smem = sizeof(la::PfSmem<D>) + 1024;

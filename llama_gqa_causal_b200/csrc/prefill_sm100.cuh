@@ -75,6 +75,7 @@ struct PrefillParams {
   int n_pb;                // ceil(S / BM)
   int n_kb;                // ceil(S / BN)
   int ctas_per_kvh;        // ceil(group * n_pb / 2)
+  int bkv_per_bundle;      // (batch, K/V head) pairs scheduled together (their K/V fit in L2)
   int causal;
   float scale_log2;        // scale * log2(e)
 };
@@ -112,10 +113,17 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  // ---- work decomposition: heavy (late position blocks) CTAs first
+  // ---- work decomposition.  The (batch, K/V head) pairs are taken in bundles
+  // whose K/V fit in L2 together, so the CTAs that share a K/V head run close
+  // in time and its tiles are read from DRAM about once; inside a bundle, heavy
+  // (late position block) CTAs go first, over all of the bundle's pairs.
   const int n_bkv = p.bsz * p.Hkv;
-  const int rank = blockIdx.x / n_bkv;
-  const int bkv = blockIdx.x - rank * n_bkv;
+  const int nb = p.bkv_per_bundle;
+  const int bundle = blockIdx.x / (nb * p.ctas_per_kvh);
+  const int bsize = min(nb, n_bkv - bundle * nb);  // the last bundle may be smaller
+  const int local = blockIdx.x - bundle * nb * p.ctas_per_kvh;
+  const int rank = local / bsize;
+  const int bkv = bundle * nb + (local - rank * bsize);
   const int b = bkv / p.Hkv, kvh = bkv - (bkv / p.Hkv) * p.Hkv;
   const int cta = p.ctas_per_kvh - 1 - rank;
   // two units per CTA, kept in scalars (never in arrays indexed at run time)

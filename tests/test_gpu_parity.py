@@ -108,6 +108,23 @@ def test_full_size_prefill_workloads_sampled(name):
     _check(out, ref, torch.bfloat16, name + " (sampled rows)", report=True)
 
 
+@pytest.mark.parametrize("name", ["llama7b", "llama70b"])
+def test_full_size_prefill_every_row_of_a_head_per_kv_group(name):
+    # every row of one query head per K/V group (the group's last head), so all
+    # position blocks, diagonal tiles and K/V heads are compared in full
+    cfg = W.PREFILL_CONFIGS[name]
+    x = W.prefill_inputs(cfg)
+    out = _gpu_prefill(cfg, x)
+    g, D = cfg.n_heads // cfg.n_kv_heads, cfg.head_dim
+    ref = np.full(out.shape, np.nan)
+    for kvh in range(cfg.n_kv_heads):
+        h = kvh * g + g - 1
+        part = oracle.prefill(x["q"], x["k"], x["v"], x["pos"], theta=cfg.theta, factor=cfg.factor,
+                              scale=cfg.scale, causal=cfg.causal, heads=(h, h + 1))
+        ref[:, :, h * D:(h + 1) * D] = part[:, :, h * D:(h + 1) * D]
+    _check(out, ref, torch.bfloat16, name + " (all rows, a head per K/V group)", report=True)
+
+
 def test_decode70b_workload():
     cfg = W.DECODE70B
     x = W.decode_inputs(cfg)  # cache tail past each length is NaN
