@@ -583,6 +583,22 @@ def run_configs(args):
                           "ms_per_call": round(ms, 5), "value": round(gbs, 1), "unit": "GB/s",
                           "frac": round(gbs / hbm, 4), "peak": f"{hbm} GB/s ({peak_src} copy)"}),
               flush=True)
+        # the same step with the new token's own key/value appended at row
+        # p = min(len, L - 1) and attended (rows 0..p); every call rewrites the
+        # same rows with the same values
+        g = torch.Generator().manual_seed(cfg.seed + 2)
+        k_new = W.normal((cfg.bsz, cfg.n_kv_heads, cfg.head_dim), cfg.dtype, g).to(dev)
+        v_new = W.normal((cfg.bsz, cfg.n_kv_heads, cfg.head_dim), cfg.dtype, g).to(dev)
+        ms = timed(lambda: api.decode_append(d["q"], k_new, v_new, d["k_cache"], d["v_cache"],
+                                             d["lens"], cos, sin, scale=cfg.scale, out=out,
+                                             workspace=wsp))
+        rows = x["lens"].to(torch.int64).clamp(0, cfg.max_cache_len - 1) + 1
+        nbytes = int(2 * rows.sum().item() * cfg.n_kv_heads * cfg.head_dim * 2)
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        print(json.dumps({"phase": "configs", "workload": cfg.name + "+append",
+                          "dtype": str(cfg.dtype).split(".")[-1], "ms_per_call": round(ms, 5),
+                          "value": round(gbs, 1), "unit": "GB/s", "frac": round(gbs / hbm, 4),
+                          "peak": f"{hbm} GB/s ({peak_src} copy)"}), flush=True)
 
 
 def main():

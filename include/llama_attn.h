@@ -128,6 +128,34 @@ int llama_attn_decode(const void* q, const void* k_cache, const void* v_cache,
                       int dtype, void* cuda_stream);
 
 /*
+ * One decode step with the new token's own key and value ("LLaMA2 large
+ * language model architecture analysis", section "KV cache": the step's key
+ * and value are appended to the cache, then the query attends over every row
+ * including its own).  For each batch entry b, with p = min(max(cache_lens[b],
+ * 0), max_cache_len - 1) the new token's row:
+ *   k_cache[b, g, p, :] = RoPE(k_new[b, g, :]) rotated with cos/sin[b] (the
+ *                         query's position, which is the new token's), rounded
+ *                         to bf16; v_cache[b, g, p, :] = v_new[b, g, :]
+ *   out[b, h*D:(h+1)*D] = attention of RoPE(q[b, h]) over cache rows 0..p of
+ *                         K/V head h / (n_heads / n_kv_heads)
+ * in one pass (no separate append launch).
+ *   q            [bsz, n_heads, head_dim], not rotated
+ *   k_new, v_new [bsz, n_kv_heads, head_dim]; k_new not rotated
+ *   k_cache, v_cache  as llama_attn_decode, written at row p (and nowhere else)
+ *   cache_lens   device int32 [bsz], read only: the caller advances it
+ *   cos, sin, out, workspace  as llama_attn_decode
+ * bf16 only.  Errors: as llama_attn_decode, plus INVALID_ARG for a NULL or
+ * misaligned k_new / v_new, and UNSUPPORTED for fp32.  A batch entry whose
+ * cache is full (cache_lens[b] >= max_cache_len) has its last row replaced.
+ */
+int llama_attn_decode_append(const void* q, const void* k_new, const void* v_new,
+                             void* k_cache, void* v_cache, const int* cache_lens,
+                             const float* cos, const float* sin, int bsz, int n_heads,
+                             int n_kv_heads, int max_cache_len, int head_dim, float scale,
+                             void* out, void* workspace, size_t workspace_bytes, int dtype,
+                             void* cuda_stream);
+
+/*
  * Single-token decode for callers that cannot allocate device memory.  The
  * pages have no counterpart to this entry point; it exists for integrations
  * that hand the library only their input and output buffers -- hosts that

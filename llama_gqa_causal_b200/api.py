@@ -36,6 +36,7 @@ EXPORTED = (
     "llama_attn_prefill",
     "llama_attn_decode_workspace_bytes",
     "llama_attn_decode",
+    "llama_attn_decode_append",
     "llama_attn_decode_noalloc",
     "llama_attn_device_status",
     "llama_attn_status_string",
@@ -81,6 +82,8 @@ def load() -> ctypes.CDLL:
     lib.llama_attn_decode_workspace_bytes.restype = Z
     lib.llama_attn_decode.argtypes = [P, P, P, P, P, P, I, I, I, I, I, F, P, P, Z, I, P]
     lib.llama_attn_decode.restype = I
+    lib.llama_attn_decode_append.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, F, P, P, Z, I, P]
+    lib.llama_attn_decode_append.restype = I
     lib.llama_attn_decode_noalloc.argtypes = [P, P, P, P, P, P, I, I, I, I, I, F, P, I, P]
     lib.llama_attn_decode_noalloc.restype = I
     lib.llama_attn_device_status.argtypes = [P]
@@ -196,6 +199,38 @@ def decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
                                  _ptr(cos), _ptr(sin), b, H, Hkv, L, D, float(scale), _ptr(out),
                                  _ptr(workspace), ws_bytes, _dtype_code(q.dtype),
                                  _stream(stream)), "llama_attn_decode")
+    return out
+
+
+def decode_append(q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor,
+                  k_cache: torch.Tensor, v_cache: torch.Tensor, cache_lens: torch.Tensor,
+                  cos: Optional[torch.Tensor] = None, sin: Optional[torch.Tensor] = None, *,
+                  scale: Optional[float] = None, out: Optional[torch.Tensor] = None,
+                  workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """llama_attn_decode_append.  q [b,H,D], k_new/v_new [b,Hkv,D] (k_new not rotated),
+    caches [b,Hkv,L,D] (written at row min(cache_lens[b], L-1)), cache_lens int32 [b]
+    (read only) -> out [b, H*D]."""
+    lib = load()
+    b, H, D = q.shape
+    Hkv, L = k_cache.shape[1], k_cache.shape[2]
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    if out is None:
+        out = torch.empty(b, H * D, device=q.device, dtype=q.dtype)
+    if workspace is None:
+        workspace = torch.empty(decode_workspace_bytes(b, H, L, D), device=q.device,
+                                dtype=torch.uint8)
+    ws_bytes = workspace.numel() * workspace.element_size()
+    if cache_lens.dtype != torch.int32:
+        raise ValueError("llama_attn_decode_append: cache_lens must be int32")
+    for name, t in (("k_new", k_new), ("v_new", v_new)):
+        if tuple(t.shape) != (b, Hkv, D) or not t.is_contiguous():
+            raise ValueError(f"llama_attn_decode_append: {name} must be contiguous [b, Hkv, D]")
+    _check(lib.llama_attn_decode_append(_ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_cache),
+                                        _ptr(v_cache), _ptr(cache_lens), _ptr(cos), _ptr(sin), b, H,
+                                        Hkv, L, D, float(scale), _ptr(out), _ptr(workspace),
+                                        ws_bytes, _dtype_code(q.dtype), _stream(stream)),
+           "llama_attn_decode_append")
     return out
 
 

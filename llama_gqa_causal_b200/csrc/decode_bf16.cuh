@@ -26,6 +26,16 @@
 // segment can start inside a sequence).  decode_combine_kernel re-derives the
 // segment boundaries from the chunk counts and merges with the log-sum-exp
 // identity.
+//
+// Append mode (the decode step's own K/V row, "LLaMA2 large language model
+// architecture analysis", section "KV cache": the new token's key and value
+// join the cache before it is attended): the new token takes row
+// p = min(len, L - 1) of its sequence; its key is rotated with the query's
+// cos/sin row (the same position), both rows are written into the caches, and
+// rows 0..p are attended.  The producer brings k_new, v_new (and cos/sin) with
+// the tile that holds row p; the consumer warp that owns the row replaces the
+// stale row in shared memory before using the tile, and the first head chunk
+// of the sequence writes the row back to the caches.
 #pragma once
 #include "common.cuh"
 
@@ -47,6 +57,10 @@ struct DecodeParams {
   const float* cos;        // [b, D] or null
   const float* sin;
   const int* lens;         // [b]
+  const __nv_bfloat16* k_new;  // append mode: [b, Hkv, D] un-rotated key of the new token
+  const __nv_bfloat16* v_new;  // append mode: [b, Hkv, D]
+  __nv_bfloat16* k_cache;      // append mode: the caches, written at row p
+  __nv_bfloat16* v_cache;
   float* ws_home;          // [b, H, D + 4]: partial of the segment at a sequence's start
   float* ws_cta;           // [MAX_CTAS, 8, D + 4]: partial of a CTA's mid-sequence segment
   int bsz, H, Hkv, L, group, hchunks;
@@ -62,6 +76,8 @@ struct DecTileMeta {
   int seg_end;     // last tile of a segment: consumers merge and write a partial
   int home;        // the segment starts at row 0 of its sequence
   int last;        // the CTA's final tile
+  int new_row;     // append mode: row of the tile that holds the new token, else -1
+  int new_pos;     // append mode: that row's index in the cache (p)
 };
 
 template <int D>
@@ -70,6 +86,7 @@ struct DecSmem {
   alignas(1024) __nv_bfloat16 v[dec::NSTAGE][dec::TR * D];
   alignas(16) __nv_bfloat16 qv[dec::NSTAGE][8 * D];  // query slice at segment starts
   alignas(16) float cs[dec::NSTAGE][2 * D];            // cos row, sin row at segment starts
+  alignas(16) __nv_bfloat16 kvn[dec::NSTAGE][2][D];    // append mode: k_new, v_new with their tile
   DecTileMeta meta[dec::NSTAGE];
   uint64_t full[dec::NSTAGE];
   uint64_t empty[dec::NSTAGE];
@@ -117,6 +134,11 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
 }
 
 __device__ __forceinline__ int clamp_len(int len, int L) { return len < 0 ? 0 : (len > L ? L : len); }
+// Rows attended: the cached rows (clamped to [0, L]), or in append mode the
+// cached rows before the new token's row p = min(len, L - 1) plus that row.
+__device__ __forceinline__ int attend_len(int len, int L, int append) {
+  return append ? clamp_len(len, L - 1) + 1 : clamp_len(len, L);
+}
 
 // Even split of n chunks over g CTAs: CTA i owns chunks [share_start(i), share_start(i + 1)).
 __device__ __forceinline__ long long share_start(long long i, long long n, long long g) {
@@ -127,7 +149,7 @@ __device__ __forceinline__ long long share_owner(long long x, long long n, long 
   return ((x + 1) * g + n - 1) / n - 1;
 }
 
-template <int D>
+template <int D, bool APPEND>
 __global__ void __launch_bounds__(dec::THREADS, 1) decode_bf16_kernel(
     const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
     DecodeParams p) {
@@ -155,7 +177,7 @@ __global__ void __launch_bounds__(dec::THREADS, 1) decode_bf16_kernel(
     const int per = (p.bsz + THREADS - 1) / THREADS;
     const int lo = min(p.bsz, static_cast<int>(threadIdx.x) * per), hi = min(p.bsz, lo + per);
     int sum = 0;
-    for (int b = lo; b < hi; ++b) sum += (clamp_len(p.lens[b], p.L) + CH - 1) / CH;
+    for (int b = lo; b < hi; ++b) sum += (attend_len(p.lens[b], p.L, APPEND) + CH - 1) / CH;
     int incl = sum;  // inclusive scan of the run totals within the warp
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -176,7 +198,7 @@ __global__ void __launch_bounds__(dec::THREADS, 1) decode_bf16_kernel(
     if (threadIdx.x == THREADS - 1) s.chunk_prefix[p.bsz] = acc + sum;
     for (int b = lo; b < hi; ++b) {
       s.chunk_prefix[b] = acc;
-      acc += (clamp_len(p.lens[b], p.L) + CH - 1) / CH;
+      acc += (attend_len(p.lens[b], p.L, APPEND) + CH - 1) / CH;
     }
     __syncthreads();
   }
@@ -200,7 +222,7 @@ __global__ void __launch_bounds__(dec::THREADS, 1) decode_bf16_kernel(
       const int seq = static_cast<int>(xb / nch_b);
       const int c = static_cast<int>(xb - static_cast<long long>(seq) * nch_b);
       const int kvh = seq / p.hchunks, hc = seq - kvh * p.hchunks;
-      const int len = clamp_len(p.lens[b], p.L);
+      const int len = attend_len(p.lens[b], p.L, APPEND);
       const bool first_chunk_of_seg = (x == x0) || (c == 0);
       const bool last_chunk_of_seg = (x + 1 == x1) || (c + 1 == nch_b);
       if (first_chunk_of_seg) home = (c == 0);
@@ -223,9 +245,16 @@ __global__ void __launch_bounds__(dec::THREADS, 1) decode_bf16_kernel(
           m.seg_end = last_chunk_of_seg && tile_last_of_chunk;
           m.home = home;
           m.last = (x + 1 == x1) && tile_last_of_chunk;
+          // append mode: the new token is the sequence's last row
+          const bool has_new = APPEND && row0 <= len - 1 && len - 1 < row0 + TR;
+          m.new_row = has_new ? len - 1 - row0 : -1;
+          m.new_pos = len - 1;
+          const bool need_cs = p.cos != nullptr && (seg_start || has_new);
           const int nh = min(8, p.group - hc * 8);
           uint32_t bytes = 2u * TR * D * 2u;
-          if (seg_start) bytes += nh * D * 2u + (p.cos != nullptr ? 2u * D * 4u : 0u);
+          if (seg_start) bytes += nh * D * 2u;
+          if (need_cs) bytes += 2u * D * 4u;
+          if (has_new) bytes += 2u * D * 2u;
           mbar_arrive_expect_tx(&s.full[st], bytes);
           const int bh = b * p.Hkv + kvh;
 #pragma unroll
@@ -233,13 +262,16 @@ __global__ void __launch_bounds__(dec::THREADS, 1) decode_bf16_kernel(
             tma_load_3d(&s.k[st][cb * TR * 64], &tm_k, &s.full[st], cb * 64, row0, bh);
             tma_load_3d(&s.v[st][cb * TR * 64], &tm_v, &s.full[st], cb * 64, row0, bh);
           }
-          if (seg_start) {
+          if (seg_start)
             bulk_load(&s.qv[st][0], p.q + (static_cast<size_t>(b) * p.H + kvh * p.group + hc * 8) * D,
                       nh * D * 2u, &s.full[st]);
-            if (p.cos != nullptr) {
-              bulk_load(&s.cs[st][0], p.cos + static_cast<size_t>(b) * D, D * 4u, &s.full[st]);
-              bulk_load(&s.cs[st][D], p.sin + static_cast<size_t>(b) * D, D * 4u, &s.full[st]);
-            }
+          if (need_cs) {
+            bulk_load(&s.cs[st][0], p.cos + static_cast<size_t>(b) * D, D * 4u, &s.full[st]);
+            bulk_load(&s.cs[st][D], p.sin + static_cast<size_t>(b) * D, D * 4u, &s.full[st]);
+          }
+          if (has_new) {
+            bulk_load(&s.kvn[st][0][0], p.k_new + static_cast<size_t>(bh) * D, D * 2u, &s.full[st]);
+            bulk_load(&s.kvn[st][1][0], p.v_new + static_cast<size_t>(bh) * D, D * 2u, &s.full[st]);
           }
         }
         __syncwarp();
@@ -296,6 +328,41 @@ __global__ void __launch_bounds__(dec::THREADS, 1) decode_bf16_kernel(
         qf[kk][0] = pack_bf16x2(y[0], y[1]);
         qf[kk][1] = pack_bf16x2(y[2], y[3]);
       }
+    }
+    if (APPEND && m.new_row >= 0 && (m.new_row >> 4) == warp) {
+      // append mode: this warp's rows hold the new token.  Replace the stale
+      // row of the stage by the rotated k_new and by v_new (same 128-byte
+      // swizzle as the TMA tile), and let the first head chunk of the sequence
+      // write both rows into the caches.
+      const int r = m.new_row;
+      uint8_t* kb = reinterpret_cast<uint8_t*>(&s.k[st][0]);
+      uint8_t* vb = reinterpret_cast<uint8_t*>(&s.v[st][0]);
+      const size_t crow = (static_cast<size_t>(m.b * p.Hkv + m.kvh) * p.L + m.new_pos) * D;
+      auto at = [&](int dd) {
+        return (dd / 64) * STAGE_BLOCK_BYTES + sw128_offset(r, (dd % 64) / 8) + (dd % 8) * 2;
+      };
+      for (int i = lane; i < D / 2; i += 32) {
+        const int d1 = i, d2 = i + D / 2;
+        const float x = __bfloat162float(s.kvn[st][0][d1]), z = __bfloat162float(s.kvn[st][0][d2]);
+        float k1 = x, k2 = z;
+        if (p.cos != nullptr) {
+          k1 = fmaf(x, s.cs[st][d1], -z * s.cs[st][D + d1]);
+          k2 = fmaf(z, s.cs[st][d2], x * s.cs[st][D + d2]);
+        }
+        const __nv_bfloat16 kr1 = __float2bfloat16_rn(k1), kr2 = __float2bfloat16_rn(k2);
+        const __nv_bfloat16 v1 = s.kvn[st][1][d1], v2 = s.kvn[st][1][d2];
+        *reinterpret_cast<__nv_bfloat16*>(kb + at(d1)) = kr1;
+        *reinterpret_cast<__nv_bfloat16*>(kb + at(d2)) = kr2;
+        *reinterpret_cast<__nv_bfloat16*>(vb + at(d1)) = v1;
+        *reinterpret_cast<__nv_bfloat16*>(vb + at(d2)) = v2;
+        if (m.hc == 0) {
+          p.k_cache[crow + d1] = kr1;
+          p.k_cache[crow + d2] = kr2;
+          p.v_cache[crow + d1] = v1;
+          p.v_cache[crow + d2] = v2;
+        }
+      }
+      __syncwarp();
     }
     const int nvalid = min(16, m.nvalid - warp * 16);
     const uint32_t kbase = smem_u32(&s.k[st][0]);
@@ -452,7 +519,7 @@ template <int D>
 __global__ void __launch_bounds__(dec::COMBINE_THREADS) decode_combine_kernel(
     const float* __restrict__ ws_home, const float* __restrict__ ws_cta,
     const int* __restrict__ lens, __nv_bfloat16* __restrict__ out, int bsz, int H, int Hkv, int L,
-    int group, int hchunks, int n_ctas) {
+    int group, int hchunks, int n_ctas, int append) {
   constexpr int kEager = 4;
   constexpr int VEC = D / 32;  // dimensions per lane
   constexpr int NW = dec::COMBINE_THREADS / 32;
@@ -463,7 +530,7 @@ __global__ void __launch_bounds__(dec::COMBINE_THREADS) decode_combine_kernel(
   __shared__ long long red[2][NW];
   long long before = 0, all = 0;
   for (int e = threadIdx.x; e < bsz; e += dec::COMBINE_THREADS) {
-    const int c = (clamp_len(lens[e], L) + dec::CH - 1) / dec::CH;
+    const int c = (attend_len(lens[e], L, append) + dec::CH - 1) / dec::CH;
     all += c;
     if (e < b) before += c;
   }
@@ -484,7 +551,7 @@ __global__ void __launch_bounds__(dec::COMBINE_THREADS) decode_combine_kernel(
     total += red[1][w];
   }
   const int per_b = Hkv * hchunks;
-  const int nch = (clamp_len(lens[b], L) + dec::CH - 1) / dec::CH;
+  const int nch = (attend_len(lens[b], L, append) + dec::CH - 1) / dec::CH;
   const long long n_chunks = total * per_b;
   const long long G = n_ctas;
   const long long P = prefix_b * per_b + static_cast<long long>(seq) * nch;

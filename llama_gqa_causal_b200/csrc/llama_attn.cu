@@ -195,7 +195,8 @@ static_assert(sizeof(la::PfSmem<128>) + 1024 <= 227 * 1024, "prefill shared memo
 template <int D>
 int decode_bf16(const void* q, const void* kc, const void* vc, const int* lens, const float* cos,
                 const float* sin, int bsz, int H, int Hkv, int L, float scale, void* out,
-                void* workspace, cudaStream_t st) {
+                void* workspace, cudaStream_t st, const void* k_new = nullptr,
+                const void* v_new = nullptr) {
   CUtensorMap tk, tv;
   const cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(L),
                               static_cast<cuuint64_t>(bsz) * Hkv};
@@ -210,6 +211,12 @@ int decode_bf16(const void* q, const void* kc, const void* vc, const int* lens, 
   p.cos = cos;
   p.sin = sin;
   p.lens = lens;
+  // append mode when the new token's rows are given: the kernel writes them
+  // into the caches (the public entry takes the caches as writable)
+  p.k_new = static_cast<const __nv_bfloat16*>(k_new);
+  p.v_new = static_cast<const __nv_bfloat16*>(v_new);
+  p.k_cache = static_cast<__nv_bfloat16*>(const_cast<void*>(kc));
+  p.v_cache = static_cast<__nv_bfloat16*>(const_cast<void*>(vc));
   p.ws_home = static_cast<float*>(workspace);
   p.ws_cta = p.ws_home + static_cast<size_t>(bsz) * H * la::dec::part_stride(D);
   p.bsz = bsz;
@@ -220,8 +227,14 @@ int decode_bf16(const void* q, const void* kc, const void* vc, const int* lens, 
   p.hchunks = (p.group + 7) / 8;
   p.scale_log2 = scale * 1.4426950408889634f;
   const size_t smem = sizeof(la::DecSmem<D>) + 1024;
-  if (!ensure_smem_attr<la::decode_bf16_kernel<D>>(smem)) return LLAMA_ERR_CUDA;
-  la::decode_bf16_kernel<D><<<n_ctas, la::dec::THREADS, smem, st>>>(tk, tv, p);
+  const int append = (k_new != nullptr) ? 1 : 0;
+  if (append) {
+    if (!ensure_smem_attr<la::decode_bf16_kernel<D, true>>(smem)) return LLAMA_ERR_CUDA;
+    la::decode_bf16_kernel<D, true><<<n_ctas, la::dec::THREADS, smem, st>>>(tk, tv, p);
+  } else {
+    if (!ensure_smem_attr<la::decode_bf16_kernel<D, false>>(smem)) return LLAMA_ERR_CUDA;
+    la::decode_bf16_kernel<D, false><<<n_ctas, la::dec::THREADS, smem, st>>>(tk, tv, p);
+  }
   if (int e = launch_status()) return e;
   // the combine launches as a programmatic dependent of the split kernel: its
   // blocks are scheduled while the split kernel drains and wait on the device
@@ -240,7 +253,8 @@ int decode_bf16(const void* q, const void* kc, const void* vc, const int* lens, 
   __nv_bfloat16* o = static_cast<__nv_bfloat16*>(out);
   int group = p.group, hchunks = p.hchunks;
   const cudaError_t e = cudaLaunchKernelEx(&cfg, la::decode_combine_kernel<D>, home, ctas,
-                                           lens, o, bsz, H, Hkv, L, group, hchunks, n_ctas);
+                                           lens, o, bsz, H, Hkv, L, group, hchunks, n_ctas,
+                                           append);
   if (e != cudaSuccess) {
     fprintf(stderr, "llama_attn: combine launch failed: %s\n", cudaGetErrorString(e));
     return LLAMA_ERR_CUDA;
@@ -390,6 +404,33 @@ int llama_attn_decode(const void* q, const void* k_cache, const void* v_cache,
                        cos, sin, nullptr, cache_lens, static_cast<float*>(out), bsz, n_heads,
                        n_kv_heads, 1, max_cache_len, 1, 0, scale, st);
 }
+
+int llama_attn_decode_append(const void* q, const void* k_new, const void* v_new,
+                             void* k_cache, void* v_cache, const int* cache_lens,
+                             const float* cos, const float* sin, int bsz, int n_heads,
+                             int n_kv_heads, int max_cache_len, int head_dim, float scale,
+                             void* out, void* workspace, size_t workspace_bytes, int dtype,
+                             void* cuda_stream) {
+  if (!q || !k_new || !v_new || !k_cache || !v_cache || !cache_lens || !out)
+    return LLAMA_ERR_INVALID_ARG;
+  if (max_cache_len < 1) return LLAMA_ERR_INVALID_ARG;
+  if (int e = check_common(bsz, n_heads, n_kv_heads, head_dim, dtype, cos, sin, scale)) return e;
+  if (!aligned16(q) || !aligned16(k_new) || !aligned16(v_new) || !aligned16(k_cache) ||
+      !aligned16(v_cache) || !aligned16(out) || !aligned16(cos) || !aligned16(sin) ||
+      !aligned16(workspace) || (reinterpret_cast<uintptr_t>(cache_lens) & 3u))
+    return LLAMA_ERR_INVALID_ARG;
+  if (dtype != LLAMA_DT_BF16) return LLAMA_ERR_UNSUPPORTED;
+  if (bsz > la::dec::MAX_BATCH) return LLAMA_ERR_UNSUPPORTED;
+  const size_t need = llama_attn_decode_workspace_bytes(bsz, n_heads, max_cache_len, head_dim);
+  if (workspace == nullptr || workspace_bytes < need) return LLAMA_ERR_INVALID_ARG;
+  cudaStream_t st = as_stream(cuda_stream);
+  if (head_dim == 128)
+    return decode_bf16<128>(q, k_cache, v_cache, cache_lens, cos, sin, bsz, n_heads, n_kv_heads,
+                            max_cache_len, scale, out, workspace, st, k_new, v_new);
+  return decode_bf16<64>(q, k_cache, v_cache, cache_lens, cos, sin, bsz, n_heads, n_kv_heads,
+                         max_cache_len, scale, out, workspace, st, k_new, v_new);
+}
+
 
 int llama_attn_decode_noalloc(const void* q, const void* k_cache, const void* v_cache,
                               const int* cache_lens, const float* cos, const float* sin, int bsz,

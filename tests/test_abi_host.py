@@ -124,6 +124,34 @@ def test_decode_rejects(lib, kw, status):
     assert _decode(lib, **kw) == status
 
 
+def _decode_append(lib, **kw):
+    a = dict(q=FAKE, kn=FAKE, vn=FAKE, kc=FAKE, vc=FAKE, lens=FAKE, cos=None, sin=None, bsz=2, H=8,
+             Hkv=2, L=100, D=128, scale=0.1, out=FAKE, ws=FAKE, ws_bytes=1 << 30, dtype=1,
+             stream=None)
+    a.update(kw)
+    return lib.llama_attn_decode_append(a["q"], a["kn"], a["vn"], a["kc"], a["vc"], a["lens"],
+                                        a["cos"], a["sin"], a["bsz"], a["H"], a["Hkv"], a["L"],
+                                        a["D"], a["scale"], a["out"], a["ws"], a["ws_bytes"],
+                                        a["dtype"], a["stream"])
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(kn=None), 1),
+    (dict(vn=None), 1),
+    (dict(kc=None), 1),
+    (dict(vn=FAKE + 4), 1),
+    (dict(kn=FAKE + 8), 1),
+    (dict(L=0), 1),
+    (dict(ws_bytes=100), 1),
+    (dict(H=8, Hkv=3), 1),
+    (dict(dtype=0), 2),
+    (dict(D=80), 2),
+    (dict(bsz=4097), 2),
+])
+def test_decode_append_rejects(lib, kw, status):
+    assert _decode_append(lib, **kw) == status
+
+
 @pytest.mark.parametrize("args", [
     (None, 1, 4, 64, 1e4, 1.0, FAKE, FAKE),
     (FAKE, 0, 4, 64, 1e4, 1.0, FAKE, FAKE),
