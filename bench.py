@@ -564,6 +564,19 @@ def run_configs(args):
                           "ms_per_call": round(ms, 5), "value": round(tflops, 2), "unit": "TFLOP/s",
                           "frac": round(tflops / peak_burst, 4),
                           "peak": f"{peak_burst} TFLOP/s ({peak_src} bf16 burst)"}), flush=True)
+        if cfg.causal and cfg.dtype == torch.bfloat16 and cfg.seq > 4096:
+            # the same workload with a 4096-key sliding window (visible pairs only)
+            window = 4096
+            pairs = sum(min(i + 1, window) for i in range(cfg.seq))
+            wflops = 4 * cfg.head_dim * pairs * cfg.n_heads * cfg.bsz
+            ms = timed(lambda: api.prefill_window(q, k, v, cos, sin, window=window, scale=cfg.scale,
+                                                  out=out, workspace=wsp))
+            tflops = wflops / (ms * 1e-3) / 1e12
+            print(json.dumps({"phase": "configs", "workload": f"{cfg.name}+window{window}",
+                              "dtype": "bfloat16", "ms_per_call": round(ms, 5),
+                              "value": round(tflops, 2), "unit": "TFLOP/s",
+                              "frac": round(tflops / peak_burst, 4),
+                              "peak": f"{peak_burst} TFLOP/s ({peak_src} bf16 burst)"}), flush=True)
         del q, k, v, out, wsp, x
     for cfg in W.DECODE_CONFIGS.values():
         if not wanted(cfg):

@@ -100,6 +100,26 @@ int llama_attn_prefill(const void* q, const void* k, const void* v, const float*
                        const float* add_mask, int dtype, void* workspace,
                        size_t workspace_bytes, void* cuda_stream);
 
+/*
+ * Causal prefill with a sliding window: query i attends to keys j with
+ * i - window < j <= i.  The flash-attention call of "`llama.py` -- LLaMA
+ * attention layer Ulysses SP adaptation" and of "[HuggingFace Transformers]
+ * LlamaAttention source walkthrough" (forward(), the flash-attention branch)
+ * passes the model's sliding_window without defining it; this is the reading
+ * used by models that set it (a window of keys ending at the query).  K/V
+ * tiles wholly before a query block's window are neither loaded nor
+ * multiplied.
+ *   window     >= 1 keys, the query's own included; window >= seq is plain
+ *              causal attention (bit-identical to llama_attn_prefill)
+ *   everything else as llama_attn_prefill with causal = 1 and no mask
+ * bf16 only.  Errors: as llama_attn_prefill, plus INVALID_ARG for window < 1,
+ * and UNSUPPORTED for fp32.
+ */
+int llama_attn_prefill_window(const void* q, const void* k, const void* v, const float* cos,
+                              const float* sin, int bsz, int n_heads, int n_kv_heads, int seq,
+                              int head_dim, float scale, int window, void* out, int dtype,
+                              void* workspace, size_t workspace_bytes, void* cuda_stream);
+
 /* Device bytes of workspace llama_attn_decode needs (split-KV partial results). */
 size_t llama_attn_decode_workspace_bytes(int bsz, int n_heads, int max_cache_len, int head_dim);
 

@@ -34,6 +34,7 @@ EXPORTED = (
     "llama_rope_table",
     "llama_attn_prefill_workspace_bytes",
     "llama_attn_prefill",
+    "llama_attn_prefill_window",
     "llama_attn_decode_workspace_bytes",
     "llama_attn_decode",
     "llama_attn_decode_append",
@@ -78,6 +79,8 @@ def load() -> ctypes.CDLL:
     lib.llama_attn_prefill_workspace_bytes.restype = Z
     lib.llama_attn_prefill.argtypes = [P, P, P, P, P, I, I, I, I, I, F, I, P, P, I, P, Z, P]
     lib.llama_attn_prefill.restype = I
+    lib.llama_attn_prefill_window.argtypes = [P, P, P, P, P, I, I, I, I, I, F, I, P, I, P, Z, P]
+    lib.llama_attn_prefill_window.restype = I
     lib.llama_attn_decode_workspace_bytes.argtypes = [I, I, I, I]
     lib.llama_attn_decode_workspace_bytes.restype = Z
     lib.llama_attn_decode.argtypes = [P, P, P, P, P, P, I, I, I, I, I, F, P, P, Z, I, P]
@@ -173,6 +176,30 @@ def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
                                   D, float(scale), int(bool(causal)), _ptr(out), _ptr(mask),
                                   _dtype_code(q.dtype), _ptr(workspace), ws_bytes,
                                   _stream(stream)), "llama_attn_prefill")
+    return out
+
+
+def prefill_window(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                   cos: Optional[torch.Tensor] = None, sin: Optional[torch.Tensor] = None, *,
+                   window: int, scale: Optional[float] = None,
+                   out: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+                   stream=None) -> torch.Tensor:
+    """llama_attn_prefill_window.  Causal; query i sees keys i - window < j <= i."""
+    lib = load()
+    b, S, H, D = q.shape
+    Hkv = k.shape[2]
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    if out is None:
+        out = torch.empty(b, S, H * D, device=q.device, dtype=q.dtype)
+    need = prefill_workspace_bytes(b, H, Hkv, S, D, q.dtype, cos is not None)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, device=q.device, dtype=torch.uint8)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib.llama_attn_prefill_window(_ptr(q), _ptr(k), _ptr(v), _ptr(cos), _ptr(sin), b, H,
+                                         Hkv, S, D, float(scale), int(window), _ptr(out),
+                                         _dtype_code(q.dtype), _ptr(workspace), ws_bytes,
+                                         _stream(stream)), "llama_attn_prefill_window")
     return out
 
 

@@ -77,6 +77,7 @@ struct PrefillParams {
   int ctas_per_kvh;        // ceil(group * n_pb / 2)
   int bkv_per_bundle;      // (batch, K/V head) pairs scheduled together (their K/V fit in L2)
   int causal;
+  int window;              // sliding-window instance: query i sees keys i - window < j <= i
   float scale_log2;        // scale * log2(e)
 };
 
@@ -93,7 +94,7 @@ struct PfSmem {
   uint32_t tmem_base;
 };
 
-template <int D>
+template <int D, bool WINDOW>
 __global__ void __launch_bounds__(pf::THREADS, 1)
     prefill_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                          const __grid_constant__ CUtensorMap tm_k,
@@ -138,6 +139,15 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
   const int nkv0 = (u0 < n_units) ? n_tiles(pb0) : 0;
   const int nkv1 = (u1 < n_units) ? n_tiles(pb1) : 0;
   const int n_max = max(nkv0, nkv1);
+  // sliding window: a unit's first K/V tile is the one holding key
+  // pb * BM - window + 1 (the window start of its first row); the CTA streams
+  // tiles j_min .. n_max - 1, the union of its units' ranges (contiguous: the
+  // two units' position blocks differ by at most one)
+  auto first_tile = [&](int pb) { return WINDOW ? max(0, pb * BM - p.window + 1) / BN : 0; };
+  const int jlo0 = first_tile(pb0);
+  const int jlo1 = nkv1 > 0 ? first_tile(pb1) : jlo0;
+  const int j_min = min(jlo0, jlo1);
+  const int n_it = n_max - j_min;  // tiles streamed
 
   // ---- setup
   if (threadIdx.x == 0) {
@@ -191,9 +201,10 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
     }
     __syncwarp();
     int k_issued = 0, v_issued = 0;
-    for (int j = 0; j < n_max; ++j) {
-      const int ks = j % KSTAGES;
-      if (j >= KSTAGES && !mbar_wait(&s.k_empty[ks], ((j / KSTAGES) - 1) & 1)) break;
+    for (int it = 0; it < n_it; ++it) {
+      const int j = j_min + it;  // K/V tile
+      const int ks = it % KSTAGES;
+      if (it >= KSTAGES && !mbar_wait(&s.k_empty[ks], ((it / KSTAGES) - 1) & 1)) break;
       if (elect_one()) {
         mbar_arrive_expect_tx(&s.k_full[ks], TILE_BYTES);
 #pragma unroll
@@ -202,9 +213,9 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
                       &s.k_full[ks], cb * 64, kvh, j * BN, b);
       }
       __syncwarp();
-      k_issued = j + 1;
-      const int vs = j % VSTAGES;
-      if (j >= VSTAGES && !mbar_wait(&s.v_empty[vs], ((j / VSTAGES) - 1) & 1)) break;
+      k_issued = it + 1;
+      const int vs = it % VSTAGES;
+      if (it >= VSTAGES && !mbar_wait(&s.v_empty[vs], ((it / VSTAGES) - 1) & 1)) break;
       if (elect_one()) {
         mbar_arrive_expect_tx(&s.v_full[vs], TILE_BYTES);
 #pragma unroll
@@ -213,7 +224,7 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
                       &s.v_full[vs], cb * 64, kvh, j * BN, b);
       }
       __syncwarp();
-      v_issued = j + 1;
+      v_issued = it + 1;
     }
     // leave no copy in flight
     mbar_wait(&s.q_loaded[0], 0);
@@ -271,9 +282,11 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
     if (ok) ok = mbar_wait(&s.k_full[0], 0);
     if (ok) {
       tc_fence_after();
-      issue_qk(0, 0);
-      commit(&s.s_full[0]);
-      if (nkv1 > 0) {
+      if (jlo0 == j_min) {
+        issue_qk(0, 0);
+        commit(&s.s_full[0]);
+      }
+      if (nkv1 > 0 && jlo1 == j_min) {
         issue_qk(1, 0);
         commit(&s.s_full[1]);
       }
@@ -287,41 +300,57 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
 #else
     auto pwait = [&](uint64_t* bar, uint32_t par) { return mbar_wait(bar, par); };
 #endif
-    auto unit_step = [&](int t, int nkv, int j, int vs) -> bool {
-      if (j >= nkv) return true;
-      if (!pwait(&s.p_lo[t], j & 1)) return false;
+    // K tile of the next streamed iteration, waited for at most once
+    auto wait_next_k = [&](int it) -> bool {
+      if (!k_ready) {
+        if (!mbar_wait(&s.k_full[(it + 1) % KSTAGES], ((it + 1) / KSTAGES) & 1)) return false;
+        k_ready = true;
+      }
+      return true;
+    };
+    // unit t over its tiles [jlo, nkv); its own tile count jj = j - jlo sets the
+    // phases of its S / P barriers
+    auto unit_step = [&](int t, int jlo, int nkv, int j, int it, int vs) -> bool {
+      if (j + 1 == jlo) {
+        // the unit starts with the next tile: its first S = Q K^T
+        if (!wait_next_k(it)) return false;
+        tc_fence_after();
+        issue_qk(t, (it + 1) % KSTAGES);
+        commit(&s.s_full[t]);
+        return true;
+      }
+      if (j < jlo || j >= nkv) return true;
+      const int jj = j - jlo;
+      if (!pwait(&s.p_lo[t], jj & 1)) return false;
       if (!v_ready) {
-        if (!mbar_wait(&s.v_full[vs], (j / VSTAGES) & 1)) return false;
+        if (!mbar_wait(&s.v_full[vs], (it / VSTAGES) & 1)) return false;
         v_ready = true;
       }
       tc_fence_after();
-      issue_pv(t, vs, j > 0, 0);
-      if (!pwait(&s.p_hi[t], j & 1)) return false;
+      issue_pv(t, vs, jj > 0, 0);
+      if (!pwait(&s.p_hi[t], jj & 1)) return false;
       tc_fence_after();
       issue_pv(t, vs, true, 1);
       if (j + 1 == nkv) {
         commit(&s.o_full[t]);
       } else {
-        if (!k_ready) {
-          if (!mbar_wait(&s.k_full[(j + 1) % KSTAGES], ((j + 1) / KSTAGES) & 1)) return false;
-          k_ready = true;
-        }
-        issue_qk(t, (j + 1) % KSTAGES);
+        if (!wait_next_k(it)) return false;
+        issue_qk(t, (it + 1) % KSTAGES);
         commit(&s.s_full[t]);
       }
       return true;
     };
-    for (int j = 0; j < n_max && ok; ++j) {
-      const int vs = j % VSTAGES;
-      const int jn = j + 1;
-      const bool next = jn < n_max;
+    for (int it = 0; it < n_it && ok; ++it) {
+      const int j = j_min + it;
+      const int vs = it % VSTAGES;
+      const bool next = it + 1 < n_it;
       v_ready = false;
       k_ready = false;
-      ok = unit_step(0, nkv0, j, vs);
-      if (ok) ok = unit_step(1, nkv1, j, vs);
+      ok = unit_step(0, jlo0, nkv0, j, it, vs);
+      if (ok && nkv1 > 0) ok = unit_step(1, jlo1, nkv1, j, it, vs);
       if (!ok) break;
       commit(&s.v_empty[vs]);
-      if (next) commit(&s.k_empty[jn % KSTAGES]);
+      if (next) commit(&s.k_empty[(it + 1) % KSTAGES]);
     }
     // every MMA this warp issued has completed before the CTA can exit
     commit(&s.mma_done);
@@ -407,8 +436,10 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
       float m_ref = -INFINITY;  // reference max (log2 units) of the exponentials
       float l_sum = 0.f;
       bool ok = true;
-      for (int j = 0; j < n_kv; ++j) {
-        if (!mbar_wait(&s.s_full[t], j & 1)) { ok = false; break; }
+      const int my_jlo = t ? jlo1 : jlo0;
+      for (int j = my_jlo; j < n_kv; ++j) {
+        const int jj = j - my_jlo;  // this unit's tile count: barrier phases
+        if (!mbar_wait(&s.s_full[t], jj & 1)) { ok = false; break; }
         tc_fence_after();
         // S in two batches: the second half is in flight while the first half's
         // max is taken
@@ -424,11 +455,13 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
         // or a mask, and any tile when scale <= 0)
         const int key0 = j * BN;
         const bool edge = (key0 + BN > p.S) || (p.causal && key0 + BN - 1 > my_pb * BM) ||
+                          (WINDOW && key0 < my_pb * BM + BM - p.window) ||
                           (mrow != nullptr) || !scale_pos;
         float rs = 0.f;
         auto tile = [&](auto edge_c) {
           constexpr bool kEdge = decltype(edge_c)::value;
           const int lim = p.causal ? min(p.S - 1, i) : p.S - 1;  // last visible key
+          const int lo = WINDOW ? i - p.window + 1 : 0;            // first visible key
           float v[BN];
           auto fill = [&](int e0) {
 #pragma unroll
@@ -439,7 +472,7 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
                 const int key = key0 + e;
                 float xv = __uint_as_float(sr[e / 32][e % 32]) * c_log2;
                 if (mrow != nullptr && key < p.S) xv = fmaf(mrow[key], 1.4426950408889634f, xv);
-                v[e] = (key <= lim) ? xv : -INFINITY;
+                v[e] = (key <= lim && key >= lo) ? xv : -INFINITY;
               }
             }
           };
@@ -490,7 +523,7 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
               fadd2(acc[2 * k], acc[2 * k + 1], acc[2 * k], acc[2 * k + 1], p0, p1);
               pk[(e % 64) / 2] = pack_bf16x2(p0, p1);
             }
-            if (h == 0 && j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+            if (h == 0 && jj > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
               // O correction before any P of this tile is released (warp-collective
               // TMEM access when any row of the warp needs it); PV_{j-1} has
               // completed: its commit preceded this tile's S
