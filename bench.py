@@ -564,6 +564,19 @@ def run_configs(args):
                           "ms_per_call": round(ms, 5), "value": round(tflops, 2), "unit": "TFLOP/s",
                           "frac": round(tflops / peak_burst, 4),
                           "peak": f"{peak_burst} TFLOP/s ({peak_src} bf16 burst)"}), flush=True)
+        if cfg.name == "llama7b":
+            # the same batch right-padded: the second entry holds about half its rows
+            lens = [cfg.seq] + [cfg.seq // 2 + 37] * (cfg.bsz - 1)
+            sl = torch.tensor(lens, dtype=torch.int32, device=dev)
+            vflops = sum(4 * cfg.head_dim * n * (n + 1) // 2 * cfg.n_heads for n in lens)
+            ms = timed(lambda: api.prefill_varlen(q, k, v, sl, cos, sin, causal=True,
+                                                  scale=cfg.scale, out=out, workspace=wsp))
+            tflops = vflops / (ms * 1e-3) / 1e12
+            print(json.dumps({"phase": "configs", "workload": f"{cfg.name}+varlen{lens}",
+                              "dtype": "bfloat16", "ms_per_call": round(ms, 5),
+                              "value": round(tflops, 2), "unit": "TFLOP/s",
+                              "frac": round(tflops / peak_burst, 4),
+                              "peak": f"{peak_burst} TFLOP/s ({peak_src} bf16 burst)"}), flush=True)
         if cfg.causal and cfg.dtype == torch.bfloat16 and cfg.seq > 4096:
             # the same workload with a 4096-key sliding window (visible pairs only)
             window = 4096

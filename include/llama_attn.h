@@ -120,6 +120,28 @@ int llama_attn_prefill_window(const void* q, const void* k, const void* v, const
                               int head_dim, float scale, int window, void* out, int dtype,
                               void* workspace, size_t workspace_bytes, void* cuda_stream);
 
+/*
+ * Prefill of a right-padded batch: batch entry b holds seq_lens[b] valid
+ * tokens at rows [0, seq_lens[b]) of the [bsz, seq, ...] tensors.  The
+ * flash-attention call of "`llama.py` -- LLaMA attention layer Ulysses SP
+ * adaptation" and of "[HuggingFace Transformers] LlamaAttention source
+ * walkthrough" (forward(), the flash-attention branch) receives the batch's
+ * attention_mask for this; here the valid lengths stand for a padding mask
+ * whose ones are a prefix of each row.  Each valid query attends only its own
+ * entry's valid keys (with causal, keys j <= i); output rows at or past
+ * seq_lens[b] are zero.  Work on padded rows is skipped tile by tile.
+ *   seq_lens   device int32 [bsz]; values are clamped to [0, seq] on the device.
+ *              Padded rows of q, k and v may hold anything, NaN included.
+ *   everything else as llama_attn_prefill (no additive mask)
+ * bf16 only.  Errors: as llama_attn_prefill, plus INVALID_ARG for a NULL or
+ * misaligned seq_lens, and UNSUPPORTED for fp32.
+ */
+int llama_attn_prefill_varlen(const void* q, const void* k, const void* v, const float* cos,
+                              const float* sin, const int* seq_lens, int bsz, int n_heads,
+                              int n_kv_heads, int seq, int head_dim, float scale, int causal,
+                              void* out, int dtype, void* workspace, size_t workspace_bytes,
+                              void* cuda_stream);
+
 /* Device bytes of workspace llama_attn_decode needs (split-KV partial results). */
 size_t llama_attn_decode_workspace_bytes(int bsz, int n_heads, int max_cache_len, int head_dim);
 

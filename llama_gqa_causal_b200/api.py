@@ -35,6 +35,7 @@ EXPORTED = (
     "llama_attn_prefill_workspace_bytes",
     "llama_attn_prefill",
     "llama_attn_prefill_window",
+    "llama_attn_prefill_varlen",
     "llama_attn_decode_workspace_bytes",
     "llama_attn_decode",
     "llama_attn_decode_append",
@@ -81,6 +82,8 @@ def load() -> ctypes.CDLL:
     lib.llama_attn_prefill.restype = I
     lib.llama_attn_prefill_window.argtypes = [P, P, P, P, P, I, I, I, I, I, F, I, P, I, P, Z, P]
     lib.llama_attn_prefill_window.restype = I
+    lib.llama_attn_prefill_varlen.argtypes = [P, P, P, P, P, P, I, I, I, I, I, F, I, P, I, P, Z, P]
+    lib.llama_attn_prefill_varlen.restype = I
     lib.llama_attn_decode_workspace_bytes.argtypes = [I, I, I, I]
     lib.llama_attn_decode_workspace_bytes.restype = Z
     lib.llama_attn_decode.argtypes = [P, P, P, P, P, P, I, I, I, I, I, F, P, P, Z, I, P]
@@ -200,6 +203,33 @@ def prefill_window(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
                                          Hkv, S, D, float(scale), int(window), _ptr(out),
                                          _dtype_code(q.dtype), _ptr(workspace), ws_bytes,
                                          _stream(stream)), "llama_attn_prefill_window")
+    return out
+
+
+def prefill_varlen(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, seq_lens: torch.Tensor,
+                   cos: Optional[torch.Tensor] = None, sin: Optional[torch.Tensor] = None, *,
+                   causal: bool = True, scale: Optional[float] = None,
+                   out: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+                   stream=None) -> torch.Tensor:
+    """llama_attn_prefill_varlen.  Right-padded batch; seq_lens int32 [b] valid rows."""
+    lib = load()
+    b, S, H, D = q.shape
+    Hkv = k.shape[2]
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    if seq_lens.dtype != torch.int32:
+        raise ValueError("llama_attn_prefill_varlen: seq_lens must be int32")
+    if out is None:
+        out = torch.empty(b, S, H * D, device=q.device, dtype=q.dtype)
+    need = prefill_workspace_bytes(b, H, Hkv, S, D, q.dtype, cos is not None)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, device=q.device, dtype=torch.uint8)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib.llama_attn_prefill_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(cos), _ptr(sin),
+                                         _ptr(seq_lens), b, H, Hkv, S, D, float(scale),
+                                         int(bool(causal)), _ptr(out), _dtype_code(q.dtype),
+                                         _ptr(workspace), ws_bytes, _stream(stream)),
+           "llama_attn_prefill_varlen")
     return out
 
 

@@ -98,7 +98,8 @@ int check_common(int bsz, int n_heads, int n_kv_heads, int head_dim, int dtype,
 template <int D>
 int prefill_bf16(const void* q, const void* k, const void* v, const float* cos, const float* sin,
                  int bsz, int H, int Hkv, int S, float scale, int causal, void* out,
-                 const float* mask, void* workspace, cudaStream_t st, int window = 0) {
+                 const float* mask, void* workspace, cudaStream_t st, int window = 0,
+                 const int* seq_lens = nullptr) {
   const void* k_src = k;
   if (cos != nullptr) {  // rotate every K row once into the workspace
     const long long n_tok = static_cast<long long>(bsz) * S;
@@ -154,18 +155,21 @@ int prefill_bf16(const void* q, const void* k, const void* v, const float* cos, 
   }
   p.causal = causal ? 1 : 0;
   p.window = window;
+  p.seq_lens = seq_lens;
   p.scale_log2 = scale * 1.4426950408889634f;
   const size_t smem = sizeof(la::PfSmem<D>) + 1024;
   const long long grid = static_cast<long long>(bsz) * Hkv * p.ctas_per_kvh;
   if (grid > 0x7fffffffLL) return LLAMA_ERR_INVALID_ARG;
+  const unsigned g = static_cast<unsigned>(grid);
   if (window > 0) {
-    if (!ensure_smem_attr<la::prefill_sm100_kernel<D, true>>(smem)) return LLAMA_ERR_CUDA;
-    la::prefill_sm100_kernel<D, true><<<static_cast<unsigned>(grid), la::pf::THREADS, smem, st>>>(
-        tq, tk, tv, to, p);
+    if (!ensure_smem_attr<la::prefill_sm100_kernel<D, true, false>>(smem)) return LLAMA_ERR_CUDA;
+    la::prefill_sm100_kernel<D, true, false><<<g, la::pf::THREADS, smem, st>>>(tq, tk, tv, to, p);
+  } else if (seq_lens != nullptr) {
+    if (!ensure_smem_attr<la::prefill_sm100_kernel<D, false, true>>(smem)) return LLAMA_ERR_CUDA;
+    la::prefill_sm100_kernel<D, false, true><<<g, la::pf::THREADS, smem, st>>>(tq, tk, tv, to, p);
   } else {
-    if (!ensure_smem_attr<la::prefill_sm100_kernel<D, false>>(smem)) return LLAMA_ERR_CUDA;
-    la::prefill_sm100_kernel<D, false><<<static_cast<unsigned>(grid), la::pf::THREADS, smem, st>>>(
-        tq, tk, tv, to, p);
+    if (!ensure_smem_attr<la::prefill_sm100_kernel<D, false, false>>(smem)) return LLAMA_ERR_CUDA;
+    la::prefill_sm100_kernel<D, false, false><<<g, la::pf::THREADS, smem, st>>>(tq, tk, tv, to, p);
   }
   return launch_status();
 }
@@ -394,6 +398,29 @@ int llama_attn_prefill_window(const void* q, const void* k, const void* v, const
                              nullptr, workspace, st, w);
   return prefill_bf16<64>(q, k, v, cos, sin, bsz, n_heads, n_kv_heads, seq, scale, 1, out, nullptr,
                           workspace, st, w);
+}
+
+int llama_attn_prefill_varlen(const void* q, const void* k, const void* v, const float* cos,
+                              const float* sin, const int* seq_lens, int bsz, int n_heads,
+                              int n_kv_heads, int seq, int head_dim, float scale, int causal,
+                              void* out, int dtype, void* workspace, size_t workspace_bytes,
+                              void* cuda_stream) {
+  if (!q || !k || !v || !out || !seq_lens) return LLAMA_ERR_INVALID_ARG;
+  if (seq < 1) return LLAMA_ERR_INVALID_ARG;
+  if (int e = check_common(bsz, n_heads, n_kv_heads, head_dim, dtype, cos, sin, scale)) return e;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(cos) ||
+      !aligned16(sin) || !aligned16(workspace) || (reinterpret_cast<uintptr_t>(seq_lens) & 3u))
+    return LLAMA_ERR_INVALID_ARG;
+  if (dtype != LLAMA_DT_BF16) return LLAMA_ERR_UNSUPPORTED;
+  const size_t need = llama_attn_prefill_workspace_bytes(bsz, n_heads, n_kv_heads, seq, head_dim,
+                                                         dtype, cos != nullptr);
+  if (need > 0 && (workspace == nullptr || workspace_bytes < need)) return LLAMA_ERR_INVALID_ARG;
+  cudaStream_t st = as_stream(cuda_stream);
+  if (head_dim == 128)
+    return prefill_bf16<128>(q, k, v, cos, sin, bsz, n_heads, n_kv_heads, seq, scale, causal, out,
+                             nullptr, workspace, st, 0, seq_lens);
+  return prefill_bf16<64>(q, k, v, cos, sin, bsz, n_heads, n_kv_heads, seq, scale, causal, out,
+                          nullptr, workspace, st, 0, seq_lens);
 }
 
 size_t llama_attn_decode_workspace_bytes(int bsz, int n_heads, int max_cache_len, int head_dim) {

@@ -78,6 +78,7 @@ struct PrefillParams {
   int bkv_per_bundle;      // (batch, K/V head) pairs scheduled together (their K/V fit in L2)
   int causal;
   int window;              // sliding-window instance: query i sees keys i - window < j <= i
+  const int* seq_lens;     // variable-length instance: [b] valid rows of each batch entry
   float scale_log2;        // scale * log2(e)
 };
 
@@ -94,7 +95,7 @@ struct PfSmem {
   uint32_t tmem_base;
 };
 
-template <int D, bool WINDOW>
+template <int D, bool WINDOW, bool VARLEN>
 __global__ void __launch_bounds__(pf::THREADS, 1)
     prefill_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                          const __grid_constant__ CUtensorMap tm_k,
@@ -133,8 +134,13 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
   const int pb0 = u0 / p.group, pb1 = u1 / p.group;
   const int head0 = kvh * p.group + (u0 - pb0 * p.group);
   const int head1 = kvh * p.group + (u1 - pb1 * p.group);
+  // variable length: batch entry b holds S_b valid rows (queries and keys); its
+  // padded rows are never attended and their outputs are zero
+  const int S_b = VARLEN ? min(max(p.seq_lens[b], 0), p.S) : p.S;
+  const int n_kb_b = VARLEN ? (S_b + BN - 1) / BN : p.n_kb;
   auto n_tiles = [&](int pb) {
-    return p.causal ? min(p.n_kb, ((pb + 1) * BM + BN - 1) / BN) : p.n_kb;
+    if (VARLEN && pb * BM >= S_b) return 0;  // every row of the Q tile is padding
+    return p.causal ? min(n_kb_b, ((pb + 1) * BM + BN - 1) / BN) : n_kb_b;
   };
   const int nkv0 = (u0 < n_units) ? n_tiles(pb0) : 0;
   const int nkv1 = (u1 < n_units) ? n_tiles(pb1) : 0;
@@ -186,11 +192,13 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
       tma_prefetch_desc(&tm_v);
       tma_prefetch_desc(&tm_out);
       // the two Q tiles (raw; rotated in shared memory by their softmax warps)
-      mbar_arrive_expect_tx(&s.q_loaded[0], TILE_BYTES);
+      if (nkv0 > 0) {
+        mbar_arrive_expect_tx(&s.q_loaded[0], TILE_BYTES);
 #pragma unroll
-      for (int cb = 0; cb < CB; ++cb)
-        tma_load_4d(reinterpret_cast<uint8_t*>(&s.q[0][0]) + cb * BLOCK_BYTES, &tm_q,
-                    &s.q_loaded[0], cb * 64, head0, pb0 * BM, b);
+        for (int cb = 0; cb < CB; ++cb)
+          tma_load_4d(reinterpret_cast<uint8_t*>(&s.q[0][0]) + cb * BLOCK_BYTES, &tm_q,
+                      &s.q_loaded[0], cb * 64, head0, pb0 * BM, b);
+      }
       if (nkv1 > 0) {
         mbar_arrive_expect_tx(&s.q_loaded[1], TILE_BYTES);
 #pragma unroll
@@ -227,7 +235,7 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
       v_issued = it + 1;
     }
     // leave no copy in flight
-    mbar_wait(&s.q_loaded[0], 0);
+    if (nkv0 > 0) mbar_wait(&s.q_loaded[0], 0);
     if (nkv1 > 0) mbar_wait(&s.q_loaded[1], 0);
     for (int j = max(0, k_issued - KSTAGES); j < k_issued; ++j)
       if (!mbar_wait(&s.k_full[j % KSTAGES], (j / KSTAGES) & 1)) break;
@@ -277,12 +285,13 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
       if (elect_one()) tc_commit(bar);
       __syncwarp();
     };
-    if (nkv0 > 0) ok = mbar_wait(&s.q_ready[0], 0);
+    ok = n_it > 0;  // (variable length: a CTA whose rows are all padding has no tile)
+    if (ok && nkv0 > 0) ok = mbar_wait(&s.q_ready[0], 0);
     if (ok && nkv1 > 0) ok = mbar_wait(&s.q_ready[1], 0);
     if (ok) ok = mbar_wait(&s.k_full[0], 0);
     if (ok) {
       tc_fence_after();
-      if (jlo0 == j_min) {
+      if (nkv0 > 0 && jlo0 == j_min) {
         issue_qk(0, 0);
         commit(&s.s_full[0]);
       }
@@ -325,6 +334,18 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
       if (!v_ready) {
         if (!mbar_wait(&s.v_full[vs], (it / VSTAGES) & 1)) return false;
         v_ready = true;
+        if (VARLEN && (j + 1) * BN > S_b) {
+          // the batch entry's last tile: its rows at or past S_b are padding
+          // (any value, NaN included); zero them so that their zero weights add
+          // exactly zero.  Rows stay contiguous under the swizzle.
+          const int r0 = S_b - j * BN;
+          uint8_t* vt = reinterpret_cast<uint8_t*>(&s.v[vs][0]);
+          for (int cb = 0; cb < CB; ++cb)
+            for (int idx = r0 * 8 + lane; idx < BN * 8; idx += 32)
+              *reinterpret_cast<uint4*>(vt + cb * BLOCK_BYTES + idx * 16) = make_uint4(0, 0, 0, 0);
+          fence_proxy_async_smem();
+          __syncwarp();
+        }
       }
       tc_fence_after();
       issue_pv(t, vs, jj > 0, 0);
@@ -346,7 +367,7 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
       const bool next = it + 1 < n_it;
       v_ready = false;
       k_ready = false;
-      ok = unit_step(0, jlo0, nkv0, j, it, vs);
+      if (nkv0 > 0) ok = unit_step(0, jlo0, nkv0, j, it, vs);
       if (ok && nkv1 > 0) ok = unit_step(1, jlo1, nkv1, j, it, vs);
       if (!ok) break;
       commit(&s.v_empty[vs]);
@@ -454,13 +475,13 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
         // or scaled + masked scores (tiles that touch the diagonal, the ragged end
         // or a mask, and any tile when scale <= 0)
         const int key0 = j * BN;
-        const bool edge = (key0 + BN > p.S) || (p.causal && key0 + BN - 1 > my_pb * BM) ||
+        const bool edge = (key0 + BN > S_b) || (p.causal && key0 + BN - 1 > my_pb * BM) ||
                           (WINDOW && key0 < my_pb * BM + BM - p.window) ||
                           (mrow != nullptr) || !scale_pos;
         float rs = 0.f;
         auto tile = [&](auto edge_c) {
           constexpr bool kEdge = decltype(edge_c)::value;
-          const int lim = p.causal ? min(p.S - 1, i) : p.S - 1;  // last visible key
+          const int lim = p.causal ? min(S_b - 1, i) : S_b - 1;  // last visible key
           const int lo = WINDOW ? i - p.window + 1 : 0;            // first visible key
           float v[BN];
           auto fill = [&](int e0) {
@@ -471,7 +492,7 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
               } else {
                 const int key = key0 + e;
                 float xv = __uint_as_float(sr[e / 32][e % 32]) * c_log2;
-                if (mrow != nullptr && key < p.S) xv = fmaf(mrow[key], 1.4426950408889634f, xv);
+                if (mrow != nullptr && key < S_b) xv = fmaf(mrow[key], 1.4426950408889634f, xv);
                 v[e] = (key <= lim && key >= lo) ? xv : -INFINITY;
               }
             }
@@ -556,6 +577,9 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
       // waits until the copy has read shared memory.
       if (ok && mbar_wait(&s.o_full[t], 0)) {
         tc_fence_after();
+        // (variable length: rows at or past S_b are padding and come out zero;
+        // select, since a padded query row may hold NaN)
+        const bool pad_row = VARLEN && i >= S_b;
         const float inv = (l_sum > 0.f) ? 1.f / l_sum : 0.f;
         uint8_t* ob = reinterpret_cast<uint8_t*>(&s.q[t][0]);
         const uint32_t row = static_cast<uint32_t>(r) * 128;
@@ -564,6 +588,9 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
           uint32_t orr[32];
           tmem_ld32(my_o + lane_off + c * 32, orr);
           tmem_ld_wait(orr);
+          if (pad_row)
+#pragma unroll
+            for (int e = 0; e < 32; ++e) orr[e] = 0u;
           const int cb = (c * 32) / 64;
 #pragma unroll
           for (int e = 0; e < 32; e += 8) {
@@ -587,6 +614,15 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
           bulk_wait_group_read0();
         }
         __syncwarp();
+      }
+    } else if (VARLEN && (t ? u1 : u0) < n_units) {
+      // variable length: every row of this Q tile is padding; its output rows are zero
+      const int i = my_pb * BM + r;
+      if (i < p.S) {
+        __nv_bfloat16* orow = p.out + (static_cast<size_t>(b) * p.S + i) * (static_cast<size_t>(p.H) * D) +
+                              static_cast<size_t>(t ? head1 : head0) * D;
+#pragma unroll
+        for (int c = 0; c < D / 8; ++c) *reinterpret_cast<uint4*>(orow + c * 8) = make_uint4(0, 0, 0, 0);
       }
     }
   }
