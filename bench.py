@@ -45,6 +45,7 @@ import time
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
+import numpy as np  # noqa: E402
 import torch  # noqa: E402
 
 from llama_gqa_causal_b200 import replicas, workloads as W  # noqa: E402
@@ -577,6 +578,32 @@ def run_configs(args):
                               "value": round(tflops, 2), "unit": "TFLOP/s",
                               "frac": round(tflops / peak_burst, 4),
                               "peak": f"{peak_burst} TFLOP/s ({peak_src} bf16 burst)"}), flush=True)
+        if cfg.name == "llama7b":
+            # the same heads with four sequences packed back to back
+            plens = [cfg.seq, cfg.seq // 2 + 37, 700, 300]
+            T = sum(plens)
+            g = torch.Generator().manual_seed(cfg.seed + 3)
+            pq = W.normal((T, cfg.n_heads, cfg.head_dim), cfg.dtype, g).to(dev)
+            pk = W.normal((T, cfg.n_kv_heads, cfg.head_dim), cfg.dtype, g).to(dev)
+            pv = W.normal((T, cfg.n_kv_heads, cfg.head_dim), cfg.dtype, g).to(dev)
+            ppos = torch.cat([torch.arange(n) for n in plens]).to(dev)
+            pc, ps = api.rope_table(ppos.view(1, -1), cfg.head_dim, cfg.theta, cfg.factor)
+            pc, ps = pc.view(T, -1), ps.view(T, -1)
+            cu = torch.tensor([0] + list(np.cumsum(plens)), dtype=torch.int32, device=dev)
+            pout = torch.empty(T, cfg.n_heads * cfg.head_dim, device=dev, dtype=cfg.dtype)
+            pws = torch.empty(api.prefill_workspace_bytes(1, cfg.n_heads, cfg.n_kv_heads, T,
+                                                          cfg.head_dim, cfg.dtype, True),
+                              device=dev, dtype=torch.uint8)
+            pflops = sum(4 * cfg.head_dim * n * (n + 1) // 2 * cfg.n_heads for n in plens)
+            ms = timed(lambda: api.prefill_packed(pq, pk, pv, cu, max(plens), pc, ps, causal=True,
+                                                  scale=cfg.scale, out=pout, workspace=pws))
+            tflops = pflops / (ms * 1e-3) / 1e12
+            print(json.dumps({"phase": "configs", "workload": f"{cfg.name}+packed{plens}",
+                              "dtype": "bfloat16", "ms_per_call": round(ms, 5),
+                              "value": round(tflops, 2), "unit": "TFLOP/s",
+                              "frac": round(tflops / peak_burst, 4),
+                              "peak": f"{peak_burst} TFLOP/s ({peak_src} bf16 burst)"}), flush=True)
+            del pq, pk, pv, pout, pws
         if cfg.causal and cfg.dtype == torch.bfloat16 and cfg.seq > 4096:
             # the same workload with a 4096-key sliding window (visible pairs only)
             window = 4096

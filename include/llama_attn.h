@@ -142,6 +142,33 @@ int llama_attn_prefill_varlen(const void* q, const void* k, const void* v, const
                               void* out, int dtype, void* workspace, size_t workspace_bytes,
                               void* cuda_stream);
 
+/*
+ * Prefill of packed sequences (the layout the flash-attention call of
+ * "`llama.py` -- LLaMA attention layer Ulysses SP adaptation" reaches once a
+ * padded batch has been unpadded): sequence s holds tokens
+ * [cu_seqlens[s], cu_seqlens[s + 1]) of the packed tensors, and each token
+ * attends only to its own sequence's tokens (with causal, those at or before
+ * it).  Every token row of out is written by its own sequence.
+ *   q            [total_tokens, n_heads, head_dim]
+ *   k, v         [total_tokens, n_kv_heads, head_dim]
+ *   cos, sin     fp32 [total_tokens, head_dim] (each token's own position) or NULL
+ *   cu_seqlens   device int32 [n_seqs + 1], non-decreasing from 0 to total_tokens;
+ *                values are clamped to [0, total_tokens] on the device
+ *   max_seqlen   >= every sequence length (longer sequences are cut to it:
+ *                their later rows are not computed)
+ *   out          [total_tokens, n_heads * head_dim]
+ *   workspace    llama_attn_prefill_workspace_bytes(1, n_heads, n_kv_heads,
+ *                total_tokens, head_dim, dtype, cos != NULL) bytes
+ * bf16 only.  Errors: as llama_attn_prefill, plus INVALID_ARG for a NULL or
+ * misaligned cu_seqlens, total_tokens < 1 or max_seqlen < 1, and UNSUPPORTED
+ * for fp32.
+ */
+int llama_attn_prefill_packed(const void* q, const void* k, const void* v, const float* cos,
+                              const float* sin, const int* cu_seqlens, int n_seqs,
+                              int total_tokens, int max_seqlen, int n_heads, int n_kv_heads,
+                              int head_dim, float scale, int causal, void* out, int dtype,
+                              void* workspace, size_t workspace_bytes, void* cuda_stream);
+
 /* Device bytes of workspace llama_attn_decode needs (split-KV partial results). */
 size_t llama_attn_decode_workspace_bytes(int bsz, int n_heads, int max_cache_len, int head_dim);
 

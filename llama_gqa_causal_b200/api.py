@@ -36,6 +36,7 @@ EXPORTED = (
     "llama_attn_prefill",
     "llama_attn_prefill_window",
     "llama_attn_prefill_varlen",
+    "llama_attn_prefill_packed",
     "llama_attn_decode_workspace_bytes",
     "llama_attn_decode",
     "llama_attn_decode_append",
@@ -84,6 +85,8 @@ def load() -> ctypes.CDLL:
     lib.llama_attn_prefill_window.restype = I
     lib.llama_attn_prefill_varlen.argtypes = [P, P, P, P, P, P, I, I, I, I, I, F, I, P, I, P, Z, P]
     lib.llama_attn_prefill_varlen.restype = I
+    lib.llama_attn_prefill_packed.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, F, I, P, I, P, Z, P]
+    lib.llama_attn_prefill_packed.restype = I
     lib.llama_attn_decode_workspace_bytes.argtypes = [I, I, I, I]
     lib.llama_attn_decode_workspace_bytes.restype = Z
     lib.llama_attn_decode.argtypes = [P, P, P, P, P, P, I, I, I, I, I, F, P, P, Z, I, P]
@@ -230,6 +233,34 @@ def prefill_varlen(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, seq_lens: 
                                          int(bool(causal)), _ptr(out), _dtype_code(q.dtype),
                                          _ptr(workspace), ws_bytes, _stream(stream)),
            "llama_attn_prefill_varlen")
+    return out
+
+
+def prefill_packed(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlens: torch.Tensor,
+                   max_seqlen: int, cos: Optional[torch.Tensor] = None,
+                   sin: Optional[torch.Tensor] = None, *, causal: bool = True,
+                   scale: Optional[float] = None, out: Optional[torch.Tensor] = None,
+                   workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """llama_attn_prefill_packed.  q [T,H,D], k/v [T,Hkv,D], cu_seqlens int32 [n+1] -> out [T, H*D]."""
+    lib = load()
+    T, H, D = q.shape
+    Hkv = k.shape[1]
+    n = cu_seqlens.numel() - 1
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    if cu_seqlens.dtype != torch.int32:
+        raise ValueError("llama_attn_prefill_packed: cu_seqlens must be int32")
+    if out is None:
+        out = torch.empty(T, H * D, device=q.device, dtype=q.dtype)
+    need = prefill_workspace_bytes(1, H, Hkv, T, D, q.dtype, cos is not None)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, device=q.device, dtype=torch.uint8)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib.llama_attn_prefill_packed(_ptr(q), _ptr(k), _ptr(v), _ptr(cos), _ptr(sin),
+                                         _ptr(cu_seqlens), n, T, int(max_seqlen), H, Hkv, D,
+                                         float(scale), int(bool(causal)), _ptr(out),
+                                         _dtype_code(q.dtype), _ptr(workspace), ws_bytes,
+                                         _stream(stream)), "llama_attn_prefill_packed")
     return out
 
 

@@ -99,10 +99,15 @@ template <int D>
 int prefill_bf16(const void* q, const void* k, const void* v, const float* cos, const float* sin,
                  int bsz, int H, int Hkv, int S, float scale, int causal, void* out,
                  const float* mask, void* workspace, cudaStream_t st, int window = 0,
-                 const int* seq_lens = nullptr) {
+                 const int* seq_lens = nullptr, const int* cu_seqlens = nullptr, int T = 0) {
+  // packed sequences: bsz sequences of at most S tokens inside tensors of T
+  // tokens, addressed as one batch entry of T rows
+  const bool packed = cu_seqlens != nullptr;
+  const long long rows = packed ? static_cast<long long>(T) : S;
+  const long long nbat = packed ? 1 : bsz;
   const void* k_src = k;
   if (cos != nullptr) {  // rotate every K row once into the workspace
-    const long long n_tok = static_cast<long long>(bsz) * S;
+    const long long n_tok = nbat * rows;
     const long long work = n_tok * Hkv * (D / 16);
     const int threads = 256;
     const int blocks = static_cast<int>(std::min<long long>((work + threads - 1) / threads, 148LL * 16));
@@ -114,20 +119,20 @@ int prefill_bf16(const void* q, const void* k, const void* v, const float* cos, 
   }
   CUtensorMap tq, tk, tv, to;
   const cuuint64_t qdims[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(H),
-                               static_cast<cuuint64_t>(S), static_cast<cuuint64_t>(bsz)};
+                               static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(nbat)};
   const cuuint64_t qstrides[3] = {static_cast<cuuint64_t>(D) * 2,
                                   static_cast<cuuint64_t>(H) * D * 2,
-                                  static_cast<cuuint64_t>(S) * H * D * 2};
+                                  static_cast<cuuint64_t>(rows) * H * D * 2};
   const cuuint32_t qbox[4] = {64, 1, static_cast<cuuint32_t>(la::pf::BM), 1};
   if (!make_map(&tq, q, 4, qdims, qstrides, qbox)) return LLAMA_ERR_CUDA;
   // out [b, S, H*D] has q's layout; each warp stores 32 rows
   const cuuint32_t obox[4] = {64, 1, 32, 1};
   if (!make_map(&to, out, 4, qdims, qstrides, obox)) return LLAMA_ERR_CUDA;
   const cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(Hkv),
-                              static_cast<cuuint64_t>(S), static_cast<cuuint64_t>(bsz)};
+                              static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(nbat)};
   const cuuint64_t strides[3] = {static_cast<cuuint64_t>(D) * 2,
                                  static_cast<cuuint64_t>(Hkv) * D * 2,
-                                 static_cast<cuuint64_t>(S) * Hkv * D * 2};
+                                 static_cast<cuuint64_t>(rows) * Hkv * D * 2};
   const cuuint32_t box[4] = {64, 1, static_cast<cuuint32_t>(la::pf::BN), 1};
   if (!make_map(&tk, k_src, 4, dims, strides, box)) return LLAMA_ERR_CUDA;
   if (!make_map(&tv, v, 4, dims, strides, box)) return LLAMA_ERR_CUDA;
@@ -156,20 +161,25 @@ int prefill_bf16(const void* q, const void* k, const void* v, const float* cos, 
   p.causal = causal ? 1 : 0;
   p.window = window;
   p.seq_lens = seq_lens;
+  p.cu_seqlens = cu_seqlens;
+  p.T = T;
   p.scale_log2 = scale * 1.4426950408889634f;
   const size_t smem = sizeof(la::PfSmem<D>) + 1024;
   const long long grid = static_cast<long long>(bsz) * Hkv * p.ctas_per_kvh;
   if (grid > 0x7fffffffLL) return LLAMA_ERR_INVALID_ARG;
   const unsigned g = static_cast<unsigned>(grid);
   if (window > 0) {
-    if (!ensure_smem_attr<la::prefill_sm100_kernel<D, true, false>>(smem)) return LLAMA_ERR_CUDA;
-    la::prefill_sm100_kernel<D, true, false><<<g, la::pf::THREADS, smem, st>>>(tq, tk, tv, to, p);
+    if (!ensure_smem_attr<la::prefill_sm100_kernel<D, true, 0>>(smem)) return LLAMA_ERR_CUDA;
+    la::prefill_sm100_kernel<D, true, 0><<<g, la::pf::THREADS, smem, st>>>(tq, tk, tv, to, p);
   } else if (seq_lens != nullptr) {
-    if (!ensure_smem_attr<la::prefill_sm100_kernel<D, false, true>>(smem)) return LLAMA_ERR_CUDA;
-    la::prefill_sm100_kernel<D, false, true><<<g, la::pf::THREADS, smem, st>>>(tq, tk, tv, to, p);
+    if (!ensure_smem_attr<la::prefill_sm100_kernel<D, false, 1>>(smem)) return LLAMA_ERR_CUDA;
+    la::prefill_sm100_kernel<D, false, 1><<<g, la::pf::THREADS, smem, st>>>(tq, tk, tv, to, p);
+  } else if (packed) {
+    if (!ensure_smem_attr<la::prefill_sm100_kernel<D, false, 2>>(smem)) return LLAMA_ERR_CUDA;
+    la::prefill_sm100_kernel<D, false, 2><<<g, la::pf::THREADS, smem, st>>>(tq, tk, tv, to, p);
   } else {
-    if (!ensure_smem_attr<la::prefill_sm100_kernel<D, false, false>>(smem)) return LLAMA_ERR_CUDA;
-    la::prefill_sm100_kernel<D, false, false><<<g, la::pf::THREADS, smem, st>>>(tq, tk, tv, to, p);
+    if (!ensure_smem_attr<la::prefill_sm100_kernel<D, false, 0>>(smem)) return LLAMA_ERR_CUDA;
+    la::prefill_sm100_kernel<D, false, 0><<<g, la::pf::THREADS, smem, st>>>(tq, tk, tv, to, p);
   }
   return launch_status();
 }
@@ -421,6 +431,30 @@ int llama_attn_prefill_varlen(const void* q, const void* k, const void* v, const
                              nullptr, workspace, st, 0, seq_lens);
   return prefill_bf16<64>(q, k, v, cos, sin, bsz, n_heads, n_kv_heads, seq, scale, causal, out,
                           nullptr, workspace, st, 0, seq_lens);
+}
+
+int llama_attn_prefill_packed(const void* q, const void* k, const void* v, const float* cos,
+                              const float* sin, const int* cu_seqlens, int n_seqs,
+                              int total_tokens, int max_seqlen, int n_heads, int n_kv_heads,
+                              int head_dim, float scale, int causal, void* out, int dtype,
+                              void* workspace, size_t workspace_bytes, void* cuda_stream) {
+  if (!q || !k || !v || !out || !cu_seqlens) return LLAMA_ERR_INVALID_ARG;
+  if (total_tokens < 1 || max_seqlen < 1) return LLAMA_ERR_INVALID_ARG;
+  if (int e = check_common(n_seqs, n_heads, n_kv_heads, head_dim, dtype, cos, sin, scale)) return e;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(cos) ||
+      !aligned16(sin) || !aligned16(workspace) || (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u))
+    return LLAMA_ERR_INVALID_ARG;
+  if (dtype != LLAMA_DT_BF16) return LLAMA_ERR_UNSUPPORTED;
+  const size_t need = llama_attn_prefill_workspace_bytes(1, n_heads, n_kv_heads, total_tokens,
+                                                         head_dim, dtype, cos != nullptr);
+  if (need > 0 && (workspace == nullptr || workspace_bytes < need)) return LLAMA_ERR_INVALID_ARG;
+  cudaStream_t st = as_stream(cuda_stream);
+  if (head_dim == 128)
+    return prefill_bf16<128>(q, k, v, cos, sin, n_seqs, n_heads, n_kv_heads, max_seqlen, scale,
+                             causal, out, nullptr, workspace, st, 0, nullptr, cu_seqlens,
+                             total_tokens);
+  return prefill_bf16<64>(q, k, v, cos, sin, n_seqs, n_heads, n_kv_heads, max_seqlen, scale, causal,
+                          out, nullptr, workspace, st, 0, nullptr, cu_seqlens, total_tokens);
 }
 
 size_t llama_attn_decode_workspace_bytes(int bsz, int n_heads, int max_cache_len, int head_dim) {

@@ -78,7 +78,9 @@ struct PrefillParams {
   int bkv_per_bundle;      // (batch, K/V head) pairs scheduled together (their K/V fit in L2)
   int causal;
   int window;              // sliding-window instance: query i sees keys i - window < j <= i
-  const int* seq_lens;     // variable-length instance: [b] valid rows of each batch entry
+  const int* seq_lens;     // padded variable-length instance: [b] valid rows of each batch entry
+  const int* cu_seqlens;   // packed instance: [b + 1] first token of each sequence
+  int T;                   // packed instance: tokens in the packed tensors
   float scale_log2;        // scale * log2(e)
 };
 
@@ -95,7 +97,7 @@ struct PfSmem {
   uint32_t tmem_base;
 };
 
-template <int D, bool WINDOW, bool VARLEN>
+template <int D, bool WINDOW, int VARLEN>
 __global__ void __launch_bounds__(pf::THREADS, 1)
     prefill_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                          const __grid_constant__ CUtensorMap tm_k,
@@ -134,9 +136,16 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
   const int pb0 = u0 / p.group, pb1 = u1 / p.group;
   const int head0 = kvh * p.group + (u0 - pb0 * p.group);
   const int head1 = kvh * p.group + (u1 - pb1 * p.group);
-  // variable length: batch entry b holds S_b valid rows (queries and keys); its
-  // padded rows are never attended and their outputs are zero
-  const int S_b = VARLEN ? min(max(p.seq_lens[b], 0), p.S) : p.S;
+  // variable length (VARLEN 1: right-padded batch; 2: packed sequences): entry
+  // b holds S_b valid rows (queries and keys).  Padded rows are never attended
+  // and their outputs are zero; in the packed layout the rows past S_b are the
+  // next sequence's, never attended and never written.  Packed sequence b
+  // starts at token tok0 of tensors with a batch extent of one.
+  const int tok0 = (VARLEN == 2) ? min(max(p.cu_seqlens[b], 0), p.T) : 0;
+  const int S_b = (VARLEN == 1)   ? min(max(p.seq_lens[b], 0), p.S)
+                  : (VARLEN == 2) ? min(max(p.cu_seqlens[b + 1] - tok0, 0), min(p.S, p.T - tok0))
+                                  : p.S;
+  const int bco = (VARLEN == 2) ? 0 : b;  // batch coordinate of the tensor maps
   const int n_kb_b = VARLEN ? (S_b + BN - 1) / BN : p.n_kb;
   auto n_tiles = [&](int pb) {
     if (VARLEN && pb * BM >= S_b) return 0;  // every row of the Q tile is padding
@@ -197,14 +206,14 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
 #pragma unroll
         for (int cb = 0; cb < CB; ++cb)
           tma_load_4d(reinterpret_cast<uint8_t*>(&s.q[0][0]) + cb * BLOCK_BYTES, &tm_q,
-                      &s.q_loaded[0], cb * 64, head0, pb0 * BM, b);
+                      &s.q_loaded[0], cb * 64, head0, tok0 + pb0 * BM, bco);
       }
       if (nkv1 > 0) {
         mbar_arrive_expect_tx(&s.q_loaded[1], TILE_BYTES);
 #pragma unroll
         for (int cb = 0; cb < CB; ++cb)
           tma_load_4d(reinterpret_cast<uint8_t*>(&s.q[1][0]) + cb * BLOCK_BYTES, &tm_q,
-                      &s.q_loaded[1], cb * 64, head1, pb1 * BM, b);
+                      &s.q_loaded[1], cb * 64, head1, tok0 + pb1 * BM, bco);
       }
     }
     __syncwarp();
@@ -218,7 +227,7 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
 #pragma unroll
         for (int cb = 0; cb < CB; ++cb)
           tma_load_4d(reinterpret_cast<uint8_t*>(&s.k[ks][0]) + cb * BLOCK_BYTES, &tm_k,
-                      &s.k_full[ks], cb * 64, kvh, j * BN, b);
+                      &s.k_full[ks], cb * 64, kvh, tok0 + j * BN, bco);
       }
       __syncwarp();
       k_issued = it + 1;
@@ -229,7 +238,7 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
 #pragma unroll
         for (int cb = 0; cb < CB; ++cb)
           tma_load_4d(reinterpret_cast<uint8_t*>(&s.v[vs][0]) + cb * BLOCK_BYTES, &tm_v,
-                      &s.v_full[vs], cb * 64, kvh, j * BN, b);
+                      &s.v_full[vs], cb * 64, kvh, tok0 + j * BN, bco);
       }
       __syncwarp();
       v_issued = it + 1;
@@ -418,8 +427,11 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
 #pragma unroll
             for (int st = 0; st < BATCH; ++st) {
               const int rr = wq * 32 + (bt * BATCH + st) * ROWS_PER_STEP + rsub;
-              const int pos = min(my_pb * BM + rr, p.S - 1);  // rows past S are zeros; any row's table is fine
-              const size_t trow = (static_cast<size_t>(b) * p.S + pos) * D;
+              // rows past S_b are discarded (zeros, padding or the next packed
+              // sequence); any of this entry's table rows serves them
+              const int pos = min(my_pb * BM + rr, S_b - 1);
+              const size_t trow = ((VARLEN == 2 ? static_cast<size_t>(tok0)
+                                                 : static_cast<size_t>(b) * p.S) + pos) * D;
               c1[st] = *reinterpret_cast<const float2*>(p.cos + trow + d);
               c2[st] = *reinterpret_cast<const float2*>(p.cos + trow + d2);
               s1[st] = *reinterpret_cast<const float2*>(p.sin + trow + d);
@@ -579,7 +591,7 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
         tc_fence_after();
         // (variable length: rows at or past S_b are padding and come out zero;
         // select, since a padded query row may hold NaN)
-        const bool pad_row = VARLEN && i >= S_b;
+        const bool pad_row = VARLEN == 1 && i >= S_b;
         const float inv = (l_sum > 0.f) ? 1.f / l_sum : 0.f;
         uint8_t* ob = reinterpret_cast<uint8_t*>(&s.q[t][0]);
         const uint32_t row = static_cast<uint32_t>(r) * 128;
@@ -603,19 +615,30 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
             *reinterpret_cast<uint4*>(ob + cb * BLOCK_BYTES + row + ((chunk ^ (r & 7)) << 4)) = w;
           }
         }
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0 && my_pb * BM + quarter * 32 < p.S) {  // the box holds a row below S
+        if (VARLEN != 2) {
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0 && my_pb * BM + quarter * 32 < p.S) {  // the box holds a row below S
 #pragma unroll
-          for (int cb = 0; cb < CB; ++cb)
-            tma_store_4d(&tm_out, ob + cb * BLOCK_BYTES + quarter * 32 * 128, cb * 64, head,
-                         my_pb * BM + quarter * 32, b);
-          bulk_commit_group();
-          bulk_wait_group_read0();
+            for (int cb = 0; cb < CB; ++cb)
+              tma_store_4d(&tm_out, ob + cb * BLOCK_BYTES + quarter * 32 * 128, cb * 64, head,
+                           my_pb * BM + quarter * 32, b);
+            bulk_commit_group();
+            bulk_wait_group_read0();
+          }
+        } else if (i < S_b) {
+          // packed: the rows past S_b belong to the next sequence, so each
+          // thread stores its own row (read back from the staged tile)
+          __nv_bfloat16* orow = p.out + (static_cast<size_t>(tok0) + i) * (static_cast<size_t>(p.H) * D) +
+                                static_cast<size_t>(head) * D;
+#pragma unroll
+          for (int c = 0; c < D / 8; ++c)
+            *reinterpret_cast<uint4*>(orow + c * 8) = *reinterpret_cast<const uint4*>(
+                ob + (c / 8) * BLOCK_BYTES + row + (((c % 8) ^ (r & 7)) << 4));
         }
         __syncwarp();
       }
-    } else if (VARLEN && (t ? u1 : u0) < n_units) {
+    } else if (VARLEN == 1 && (t ? u1 : u0) < n_units) {
       // variable length: every row of this Q tile is padding; its output rows are zero
       const int i = my_pb * BM + r;
       if (i < p.S) {

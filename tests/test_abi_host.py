@@ -173,6 +173,32 @@ def test_prefill_varlen_rejects(lib, kw, status):
     assert _prefill_varlen(lib, **kw) == status
 
 
+def _prefill_packed(lib, **kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, cos=None, sin=None, cu=FAKE, n=3, T=300, maxlen=128, H=8,
+             Hkv=2, D=128, scale=0.1, causal=1, out=FAKE, dtype=1, ws=None, ws_bytes=0,
+             stream=None)
+    a.update(kw)
+    return lib.llama_attn_prefill_packed(a["q"], a["k"], a["v"], a["cos"], a["sin"], a["cu"],
+                                         a["n"], a["T"], a["maxlen"], a["H"], a["Hkv"], a["D"],
+                                         a["scale"], a["causal"], a["out"], a["dtype"], a["ws"],
+                                         a["ws_bytes"], a["stream"])
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(cu=None), 1),
+    (dict(cu=FAKE + 2), 1),
+    (dict(T=0), 1),
+    (dict(maxlen=0), 1),
+    (dict(n=0), 1),
+    (dict(H=8, Hkv=3), 1),
+    (dict(cos=FAKE, sin=FAKE), 1),        # RoPE needs the K-rotation workspace
+    (dict(dtype=0), 2),
+    (dict(D=96), 2),
+])
+def test_prefill_packed_rejects(lib, kw, status):
+    assert _prefill_packed(lib, **kw) == status
+
+
 def _decode_append(lib, **kw):
     a = dict(q=FAKE, kn=FAKE, vn=FAKE, kc=FAKE, vc=FAKE, lens=FAKE, cos=None, sin=None, bsz=2, H=8,
              Hkv=2, L=100, D=128, scale=0.1, out=FAKE, ws=FAKE, ws_bytes=1 << 30, dtype=1,
