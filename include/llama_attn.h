@@ -18,6 +18,17 @@
  *   (obsidian-quartz-blog), section "KV cache": one query row per sequence
  *   attends to every cached key; nothing is masked.
  *
+ * Entry points:
+ *   llama_rope_table            cos/sin tables from positions (theta, linear factor)
+ *   llama_attn_prefill          full-sequence attention (causal or not, optional mask)
+ *   llama_attn_prefill_window   causal prefill with a sliding window
+ *   llama_attn_prefill_varlen   prefill of a right-padded batch (per-entry lengths)
+ *   llama_attn_prefill_packed   prefill of packed sequences (cu_seqlens offsets)
+ *   llama_attn_decode           one query token per sequence against a KV cache
+ *   llama_attn_decode_append    the same step with the token's own K/V appended
+ *   llama_attn_decode_noalloc   decode on a static scratch (no caller workspace)
+ *   plus workspace sizes, the device status word, status strings, ABI version.
+ *
  * Conventions shared by every entry point:
  *   - All tensor pointers are DEVICE pointers, contiguous, row-major, owned by
  *     the caller, and must be 16-byte aligned.  The library never allocates
@@ -259,7 +270,7 @@ int llama_attn_device_status(void* cuda_stream);
 /* Static, NUL-terminated description of a status code. */
 const char* llama_attn_status_string(int status);
 
-/* ABI version (major * 100 + minor). */
+/* ABI version (major * 100 + minor): 110 = 1.1, the entry points above. */
 int llama_attn_abi_version(void);
 
 #ifdef __cplusplus

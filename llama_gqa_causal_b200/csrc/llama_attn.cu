@@ -18,7 +18,7 @@
 
 namespace {
 
-constexpr int kAbiVersion = 100;
+constexpr int kAbiVersion = 110;
 
 // ---------------------------------------------------------------- host helpers
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }

@@ -33,6 +33,15 @@
 // same tcgen05 issue order, so the overwrite follows the read.
 // Rescaling of O is lazy: the running max used for the exponentials moves
 // only when a row's max grows by more than 2^8, which keeps O corrections rare.
+// Epilogue: O / l in bf16 is staged in the Q tile buffer and stored by TMA.
+//
+// Instances (template flags, so each compiles only its own bookkeeping):
+//   WINDOW          causal sliding window: a unit starts at the K/V tile of its
+//                   first row's window start; window-edge tiles are masked
+//   VARLEN == 1     right-padded batch: per-entry lengths; padded keys masked,
+//                   padded V rows zeroed in the stage, padded rows output zero
+//   VARLEN == 2     packed sequences: as 1, with each sequence addressed from
+//                   its first token and its rows stored by their own threads
 #pragma once
 #include <type_traits>
 

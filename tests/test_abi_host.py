@@ -41,7 +41,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_abi_version_and_status_strings(lib):
-    assert lib.llama_attn_abi_version() == 100
+    assert lib.llama_attn_abi_version() == 110
     assert api.status_string(0) == "ok"
     assert "invalid" in api.status_string(1)
     assert "unsupported" in api.status_string(2)
