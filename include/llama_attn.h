@@ -20,6 +20,7 @@
  *
  * Entry points:
  *   llama_rope_table            cos/sin tables from positions (theta, linear factor)
+ *   llama_rope_table_ntk        the same with NTK-aware base scaling
  *   llama_attn_prefill          full-sequence attention (causal or not, optional mask)
  *   llama_attn_prefill_window   causal prefill with a sliding window
  *   llama_attn_prefill_varlen   prefill of a right-padded batch (per-entry lengths)
@@ -80,6 +81,20 @@ typedef enum {
  */
 int llama_rope_table(const long long* pos, int bsz, int seq, int head_dim, double theta,
                      double pos_scale_factor, float* cos, float* sin, void* cuda_stream);
+
+/*
+ * RoPE table with NTK-aware scaling: as llama_rope_table with no position
+ * scaling and the base raised to theta * alpha^(head_dim / (head_dim - 2)),
+ * which keeps the highest frequency and divides the lowest by exactly alpha.
+ * "Llama2 Transformer architecture and optimisation practice" section 6.1
+ * names adjusting the base frequency for longer contexts without a formula;
+ * this is the published NTK-aware rule.  The tables feed every attention entry
+ * point unchanged.
+ * Errors: as llama_rope_table, plus INVALID_ARG for alpha <= 0, head_dim < 4
+ * or a base that overflows.
+ */
+int llama_rope_table_ntk(const long long* pos, int bsz, int seq, int head_dim, double theta,
+                         double alpha, float* cos, float* sin, void* cuda_stream);
 
 /* Device bytes of workspace llama_attn_prefill needs for this shape (0 when
  * no RoPE or dtype is fp32).  has_rope: whether cos/sin will be passed. */

@@ -32,6 +32,7 @@ LLAMA_ERR_DEVICE_TIMEOUT = 4
 # Every symbol include/llama_attn.h declares.
 EXPORTED = (
     "llama_rope_table",
+    "llama_rope_table_ntk",
     "llama_attn_prefill_workspace_bytes",
     "llama_attn_prefill",
     "llama_attn_prefill_window",
@@ -77,6 +78,8 @@ def load() -> ctypes.CDLL:
     P, I, D, Z, F = ctypes.c_void_p, ctypes.c_int, ctypes.c_double, ctypes.c_size_t, ctypes.c_float
     lib.llama_rope_table.argtypes = [P, I, I, I, D, D, P, P, P]
     lib.llama_rope_table.restype = I
+    lib.llama_rope_table_ntk.argtypes = [P, I, I, I, D, D, P, P, P]
+    lib.llama_rope_table_ntk.restype = I
     lib.llama_attn_prefill_workspace_bytes.argtypes = [I, I, I, I, I, I, I]
     lib.llama_attn_prefill_workspace_bytes.restype = Z
     lib.llama_attn_prefill.argtypes = [P, P, P, P, P, I, I, I, I, I, F, I, P, P, I, P, Z, P]
@@ -149,6 +152,21 @@ def rope_table(pos: torch.Tensor, head_dim: int, theta: float = 10000.0,
     seq = n // bsz
     _check(lib.llama_rope_table(_ptr(pos), bsz, seq, head_dim, float(theta), float(factor),
                                 _ptr(cos), _ptr(sin), _stream(stream)), "llama_rope_table")
+    return cos, sin
+
+
+def rope_table_ntk(pos: torch.Tensor, head_dim: int, theta: float = 10000.0, alpha: float = 1.0,
+                   stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """cos, sin of the NTK-aware scaled table (llama_rope_table_ntk)."""
+    lib = load()
+    pos = pos.to(torch.int64).contiguous()
+    n = pos.numel()
+    cos = torch.empty(*pos.shape, head_dim, device=pos.device, dtype=torch.float32)
+    sin = torch.empty_like(cos)
+    bsz = pos.shape[0] if pos.dim() > 1 else 1
+    seq = n // bsz
+    _check(lib.llama_rope_table_ntk(_ptr(pos), bsz, seq, head_dim, float(theta), float(alpha),
+                                    _ptr(cos), _ptr(sin), _stream(stream)), "llama_rope_table_ntk")
     return cos, sin
 
 

@@ -6,6 +6,7 @@
 #include <stdio.h>
 
 #include <algorithm>
+#include <cmath>
 #include <mutex>
 
 #include "llama_attn.h"
@@ -337,12 +338,25 @@ int llama_rope_table(const long long* pos, int bsz, int seq, int head_dim, doubl
   if (bsz < 1 || seq < 1 || head_dim < 2 || (head_dim % 2)) return LLAMA_ERR_INVALID_ARG;
   if (!(theta > 0.0) || !(pos_scale_factor > 0.0)) return LLAMA_ERR_INVALID_ARG;
   const long long n = static_cast<long long>(bsz) * seq;
-  const long long work = n * (head_dim / 2);
-  const int threads = 256;
-  const int blocks = static_cast<int>(std::min<long long>((work + threads - 1) / threads, 148LL * 32));
+  // a multiple of head_dim / 2 threads per block (one frequency index each)
+  const int half = head_dim / 2;
+  const int threads = half >= 256 ? half : (256 / half) * half;
+  const long long rows_per_block = threads / half;
+  const int blocks =
+      static_cast<int>(std::min<long long>((n + rows_per_block - 1) / rows_per_block, 148LL * 32));
+  if (threads > 1024) return LLAMA_ERR_UNSUPPORTED;
   la::rope_table_kernel<<<blocks, threads, 0, as_stream(cuda_stream)>>>(
       pos, n, head_dim, theta, pos_scale_factor, cos, sin);
   return launch_status();
+}
+
+int llama_rope_table_ntk(const long long* pos, int bsz, int seq, int head_dim, double theta,
+                         double alpha, float* cos, float* sin, void* cuda_stream) {
+  if (head_dim < 4 || !(alpha > 0.0)) return LLAMA_ERR_INVALID_ARG;
+  // the NTK-aware base theta * alpha^(D / (D - 2)), then the plain table
+  const double base = theta * std::pow(alpha, static_cast<double>(head_dim) / (head_dim - 2));
+  if (!std::isfinite(base)) return LLAMA_ERR_INVALID_ARG;
+  return llama_rope_table(pos, bsz, seq, head_dim, base, 1.0, cos, sin, cuda_stream);
 }
 
 size_t llama_attn_prefill_workspace_bytes(int bsz, int n_heads, int n_kv_heads, int seq,

@@ -19,14 +19,14 @@ namespace la {
 __global__ void rope_table_kernel(const long long* __restrict__ pos, long long n_rows, int D,
                                   double theta, double factor, float* __restrict__ cos_out,
                                   float* __restrict__ sin_out) {
+  // blockDim.x is a multiple of D/2: each thread keeps one frequency index i
+  // (so its inverse frequency is formed once) and walks the rows
   const int half = D / 2;
-  const long long total = n_rows * half;
-  const double log_theta = log(theta);
-  for (long long idx = blockIdx.x * (long long)blockDim.x + threadIdx.x; idx < total;
-       idx += (long long)gridDim.x * blockDim.x) {
-    const long long r = idx / half;
-    const int i = static_cast<int>(idx - r * half);
-    const double inv_freq = exp(-(2.0 * i / D) * log_theta);
+  const int i = static_cast<int>(threadIdx.x % half);
+  const int rows_per_block = static_cast<int>(blockDim.x / half);
+  const double inv_freq = exp(-(2.0 * i / D) * log(theta));
+  for (long long r = blockIdx.x * (long long)rows_per_block + threadIdx.x / half; r < n_rows;
+       r += (long long)gridDim.x * rows_per_block) {
     const double angle = (static_cast<double>(pos[r]) / factor) * inv_freq;
     double s, c;
     sincos(angle, &s, &c);

@@ -55,6 +55,8 @@ def _bind(path: str):
     L = ctypes.c_long
     lib.oracle_rope_cos_sin.argtypes = [P, L, I, D, D, P, P]
     lib.oracle_rope_cos_sin.restype = None
+    lib.oracle_rope_ntk_theta.argtypes = [D, D, I]
+    lib.oracle_rope_ntk_theta.restype = D
     lib.oracle_rope_rotate.argtypes = [P, L, I, P, P, P]
     lib.oracle_rope_rotate.restype = None
     lib.oracle_prefill.argtypes = [P, P, P, P, I, I, I, I, I, D, D, D, I, P,
@@ -105,6 +107,17 @@ def rope_cos_sin(pos, head_dim: int, theta: float = 10000.0, factor: float = 1.0
     s = np.empty((n, head_dim), np.float64)
     lib.oracle_rope_cos_sin(_ptr(p), n, head_dim, float(theta), float(factor), _ptr(c), _ptr(s))
     return c, s
+
+
+def rope_ntk_theta(theta: float, alpha: float, head_dim: int) -> float:
+    """Base of the NTK-aware scaled table: theta * alpha^(D / (D - 2))."""
+    lib = _load()
+    return float(lib.oracle_rope_ntk_theta(float(theta), float(alpha), int(head_dim)))
+
+
+def rope_cos_sin_ntk(pos, head_dim: int, theta: float = 10000.0, alpha: float = 1.0):
+    """cos, sin [n, head_dim] float64 of the NTK-aware scaled table."""
+    return rope_cos_sin(pos, head_dim, rope_ntk_theta(theta, alpha, head_dim), 1.0)
 
 
 def rope_rotate(x, cos, sin):

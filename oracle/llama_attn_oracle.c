@@ -58,6 +58,16 @@ void oracle_rope_cos_sin(const long long* pos, long n, int D, double theta,
   }
 }
 
+/* NTK-aware RoPE scaling: the base is raised to theta * alpha^(D / (D - 2)),
+ * so the highest frequency (i = 0) is kept and the lowest (i = D/2 - 1) is
+ * divided by exactly alpha.  [P5] 6.1 names "adjusting the base frequency" for
+ * length extrapolation without a formula; this is the published NTK-aware
+ * rule, taken as the reading.  The table is then oracle_rope_cos_sin with
+ * this base and no position scaling. */
+double oracle_rope_ntk_theta(double theta, double alpha, int D) {
+  return theta * pow(alpha, (double)D / (double)(D - 2));
+}
+
 /* y = x * cos + rotate_half(x) * sin, with rotate_half(x) = [-x[D/2:], x[:D/2]]
  * (rotate-half form of [P5] 2.1 / the apply_rotary_pos_emb of [HF] step 3). */
 void oracle_rope_rotate(const double* x, long n, int D, const double* cos_t,

@@ -199,6 +199,17 @@ def test_prefill_packed_rejects(lib, kw, status):
     assert _prefill_packed(lib, **kw) == status
 
 
+@pytest.mark.parametrize("args", [
+    (FAKE, 1, 4, 64, 1e4, 0.0, FAKE, FAKE),    # alpha must be positive
+    (FAKE, 1, 4, 64, 1e4, -2.0, FAKE, FAKE),
+    (FAKE, 1, 4, 2, 1e4, 2.0, FAKE, FAKE),     # head_dim 2 has no D - 2
+    (None, 1, 4, 64, 1e4, 2.0, FAKE, FAKE),
+    (FAKE, 1, 4, 64, 1e300, 1e300, FAKE, FAKE),  # base overflows
+])
+def test_rope_table_ntk_rejects(lib, args):
+    assert lib.llama_rope_table_ntk(*args, None) == 1
+
+
 def _decode_append(lib, **kw):
     a = dict(q=FAKE, kn=FAKE, vn=FAKE, kc=FAKE, vc=FAKE, lens=FAKE, cos=None, sin=None, bsz=2, H=8,
              Hkv=2, L=100, D=128, scale=0.1, out=FAKE, ws=FAKE, ws_bytes=1 << 30, dtype=1,

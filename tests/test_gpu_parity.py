@@ -74,6 +74,16 @@ def test_rope_table_matches_oracle(D, factor):
     assert np.abs(sin[0].cpu().double().numpy() - s).max() < 2e-7
 
 
+@pytest.mark.parametrize("D,alpha", [(128, 1.0), (128, 4.0), (64, 8.0)])
+def test_rope_table_ntk_matches_oracle(D, alpha):
+    pos = torch.cat([torch.arange(0, 8192), torch.randint(0, 1 << 17, (512,),
+                                                          generator=torch.Generator().manual_seed(2))])
+    cos, sin = api.rope_table_ntk(pos.view(1, -1).cuda(), D, 10000.0, alpha)
+    c, s = oracle.rope_cos_sin_ntk(pos.numpy(), D, 10000.0, alpha)
+    assert np.abs(cos[0].cpu().double().numpy() - c).max() < 2e-7
+    assert np.abs(sin[0].cpu().double().numpy() - s).max() < 2e-7
+
+
 # ----------------------------------------------------------------------------- named workloads
 
 def test_tiny_fp32_workload():

@@ -425,3 +425,39 @@ def test_planted_mistake_in_oracle_is_caught(mutation, tmp_path):
 
 def test_unmutated_oracle_passes_pin_suite():
     assert _pin_suite() == []
+
+
+
+# ----------------------------------------------------------------------------- NTK-aware scaling
+# The pages name adjusting the RoPE base for longer contexts without a formula;
+# the oracle takes the published NTK-aware rule.  What the rule is for fixes
+# it: alpha = 1 is the plain table, the highest frequency (i = 0) never moves,
+# and the lowest (i = D/2 - 1) is exactly linear position interpolation by alpha.
+
+@pytest.mark.parametrize("D", [64, 128])
+def test_ntk_alpha_one_is_the_plain_table(D):
+    pos = np.arange(0, 5000, 7)
+    c0, s0 = oracle.rope_cos_sin(pos, D, 10000.0, 1.0)
+    c1, s1 = oracle.rope_cos_sin_ntk(pos, D, 10000.0, 1.0)
+    assert np.array_equal(c0, c1) and np.array_equal(s0, s1)
+
+
+@pytest.mark.parametrize("D,alpha", [(64, 2.0), (128, 4.0), (128, 8.0)])
+def test_ntk_keeps_the_highest_frequency(D, alpha):
+    pos = np.arange(0, 40000, 13)
+    c0, s0 = oracle.rope_cos_sin(pos, D, 10000.0, 1.0)
+    c1, s1 = oracle.rope_cos_sin_ntk(pos, D, 10000.0, alpha)
+    assert np.array_equal(c0[:, 0], c1[:, 0]) and np.array_equal(s0[:, 0], s1[:, 0])
+
+
+@pytest.mark.parametrize("D,alpha", [(64, 2.0), (128, 4.0), (128, 8.0)])
+def test_ntk_lowest_frequency_is_linear_interpolation(D, alpha):
+    pos = np.arange(0, 40000, 13)
+    lo = D // 2 - 1
+    c_lin, s_lin = oracle.rope_cos_sin(pos, D, 10000.0, alpha)   # positions / alpha
+    c_ntk, s_ntk = oracle.rope_cos_sin_ntk(pos, D, 10000.0, alpha)
+    assert np.abs(c_ntk[:, lo] - c_lin[:, lo]).max() < 1e-9
+    assert np.abs(s_ntk[:, lo] - s_lin[:, lo]).max() < 1e-9
+    # and it is not plain interpolation elsewhere: a middle frequency moves less
+    mid = D // 4
+    assert np.abs(c_ntk[:, mid] - c_lin[:, mid]).max() > 1e-3
