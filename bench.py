@@ -629,6 +629,35 @@ def run_configs(args):
                               "value": round(nbytes / (ms * 1e-3) / 1e9, 1), "unit": "GB/s",
                               "frac": round(nbytes / (ms * 1e-3) / 1e9 / hbm, 4),
                               "peak": f"{hbm} GB/s ({peak_src} copy)"}), flush=True)
+        if cfg.name == "llama70b":
+            # the projections around the attention of this shape (hidden 8192):
+            # q/k/v with RoPE in the GEMM epilogue, then the output projection
+            hidden = cfg.n_heads * cfg.head_dim
+            n_qkv = (cfg.n_heads + 2 * cfg.n_kv_heads) * cfg.head_dim
+            T = cfg.bsz * cfg.seq
+            g = torch.Generator().manual_seed(cfg.seed + 4)
+            px = W.normal((T, hidden), cfg.dtype, g).to(dev)
+            pw = (torch.randn(n_qkv, hidden, generator=g) / hidden ** 0.5).to(cfg.dtype).to(dev)
+            pwo = (torch.randn(hidden, hidden, generator=g) / hidden ** 0.5).to(cfg.dtype).to(dev)
+            bufs = (torch.empty(T, cfg.n_heads, cfg.head_dim, device=dev, dtype=cfg.dtype),
+                    torch.empty(T, cfg.n_kv_heads, cfg.head_dim, device=dev, dtype=cfg.dtype),
+                    torch.empty(T, cfg.n_kv_heads, cfg.head_dim, device=dev, dtype=cfg.dtype))
+            ct, st_ = cos.view(T, -1), sin.view(T, -1)
+            ms = timed(lambda: api.qkv_rope(px, pw, cfg.n_heads, cfg.n_kv_heads, cfg.head_dim, ct,
+                                            st_, out=bufs))
+            tf = 2.0 * T * hidden * n_qkv / (ms * 1e-3) / 1e12
+            print(json.dumps({"phase": "configs", "workload": f"{cfg.name}+qkv_rope_proj",
+                              "dtype": "bfloat16", "ms_per_call": round(ms, 5), "value": round(tf, 2),
+                              "unit": "TFLOP/s", "frac": round(tf / peak_burst, 4),
+                              "peak": f"{peak_burst} TFLOP/s ({peak_src} bf16 burst)"}), flush=True)
+            py = torch.empty(T, hidden, device=dev, dtype=cfg.dtype)
+            ms = timed(lambda: api.out_proj(bufs[0].view(T, hidden), pwo, out=py))
+            tf = 2.0 * T * hidden * hidden / (ms * 1e-3) / 1e12
+            print(json.dumps({"phase": "configs", "workload": f"{cfg.name}+out_proj",
+                              "dtype": "bfloat16", "ms_per_call": round(ms, 5), "value": round(tf, 2),
+                              "unit": "TFLOP/s", "frac": round(tf / peak_burst, 4),
+                              "peak": f"{peak_burst} TFLOP/s ({peak_src} bf16 burst)"}), flush=True)
+            del px, pw, pwo, bufs, py
         if cfg.causal and cfg.dtype == torch.bfloat16 and cfg.seq > 4096:
             # the same workload with a 4096-key sliding window (visible pairs only)
             window = 4096

@@ -21,6 +21,8 @@
  * Entry points:
  *   llama_rope_table            cos/sin tables from positions (theta, linear factor)
  *   llama_rope_table_ntk        the same with NTK-aware base scaling
+ *   llama_attn_qkv_rope         q/k/v projection GEMM with RoPE in its epilogue
+ *   llama_attn_out_proj         output projection GEMM
  *   llama_attn_prefill          full-sequence attention (causal or not, optional mask)
  *   llama_attn_prefill_window   causal prefill with a sliding window
  *   llama_attn_prefill_varlen   prefill of a right-padded batch (per-entry lengths)
@@ -95,6 +97,39 @@ int llama_rope_table(const long long* pos, int bsz, int seq, int head_dim, doubl
  */
 int llama_rope_table_ntk(const long long* pos, int bsz, int seq, int head_dim, double theta,
                          double alpha, float* cos, float* sin, void* cuda_stream);
+
+/*
+ * Q/K/V projection with RoPE in the GEMM epilogue ("[HuggingFace Transformers]
+ * LlamaAttention source walkthrough", section 2 forward() steps 1-3: project,
+ * view per head, rotate q and k).  One tcgen05 GEMM x . w_qkv^T whose output
+ * columns are the heads of q, k and v; q and k heads are rotated with the
+ * token's cos/sin row before they are stored, so the results feed the
+ * attention entry points with cos = sin = NULL.
+ *   x        bf16 [tokens, hidden]
+ *   w_qkv    bf16 [(n_heads + 2 n_kv_heads) head_dim, hidden]: the rows of
+ *            W_q, then W_k, then W_v (the nn.Linear weight layout)
+ *   cos, sin fp32 [tokens, head_dim] (llama_rope_table of the tokens'
+ *            positions) or both NULL (no rotation)
+ *   q        bf16 [tokens, n_heads, head_dim]; k, v bf16 [tokens, n_kv_heads, head_dim]
+ * bf16 only.  Errors: INVALID_ARG for a NULL or misaligned pointer, tokens or
+ * hidden < 1, hidden not a multiple of 8, a bad head split; UNSUPPORTED for
+ * fp32 or head_dim other than 64 / 128.
+ */
+int llama_attn_qkv_rope(const void* x, const void* w_qkv, const float* cos, const float* sin,
+                        int tokens, int hidden, int n_heads, int n_kv_heads, int head_dim,
+                        void* q, void* k, void* v, int dtype, void* cuda_stream);
+
+/*
+ * Output projection y = attn . w_o^T (section 2 forward() step 7, o_proj) on
+ * the same tcgen05 GEMM with a plain epilogue.
+ *   attn     bf16 [tokens, in_dim] (the attention output, heads concatenated)
+ *   w_o      bf16 [out_dim, in_dim]
+ *   y        bf16 [tokens, out_dim]
+ * bf16 only.  Errors: INVALID_ARG for a NULL or misaligned pointer, a size < 1
+ * or in_dim / out_dim not a multiple of 8; UNSUPPORTED for fp32.
+ */
+int llama_attn_out_proj(const void* attn, const void* w_o, int tokens, int in_dim, int out_dim,
+                        void* y, int dtype, void* cuda_stream);
 
 /* Device bytes of workspace llama_attn_prefill needs for this shape (0 when
  * no RoPE or dtype is fp32).  has_rope: whether cos/sin will be passed. */

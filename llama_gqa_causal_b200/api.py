@@ -33,6 +33,8 @@ LLAMA_ERR_DEVICE_TIMEOUT = 4
 EXPORTED = (
     "llama_rope_table",
     "llama_rope_table_ntk",
+    "llama_attn_qkv_rope",
+    "llama_attn_out_proj",
     "llama_attn_prefill_workspace_bytes",
     "llama_attn_prefill",
     "llama_attn_prefill_window",
@@ -80,6 +82,10 @@ def load() -> ctypes.CDLL:
     lib.llama_rope_table.restype = I
     lib.llama_rope_table_ntk.argtypes = [P, I, I, I, D, D, P, P, P]
     lib.llama_rope_table_ntk.restype = I
+    lib.llama_attn_qkv_rope.argtypes = [P, P, P, P, I, I, I, I, I, P, P, P, I, P]
+    lib.llama_attn_qkv_rope.restype = I
+    lib.llama_attn_out_proj.argtypes = [P, P, I, I, I, P, I, P]
+    lib.llama_attn_out_proj.restype = I
     lib.llama_attn_prefill_workspace_bytes.argtypes = [I, I, I, I, I, I, I]
     lib.llama_attn_prefill_workspace_bytes.restype = Z
     lib.llama_attn_prefill.argtypes = [P, P, P, P, P, I, I, I, I, I, F, I, P, P, I, P, Z, P]
@@ -168,6 +174,39 @@ def rope_table_ntk(pos: torch.Tensor, head_dim: int, theta: float = 10000.0, alp
     _check(lib.llama_rope_table_ntk(_ptr(pos), bsz, seq, head_dim, float(theta), float(alpha),
                                     _ptr(cos), _ptr(sin), _stream(stream)), "llama_rope_table_ntk")
     return cos, sin
+
+
+def qkv_rope(x: torch.Tensor, w_qkv: torch.Tensor, n_heads: int, n_kv_heads: int, head_dim: int,
+             cos: Optional[torch.Tensor] = None, sin: Optional[torch.Tensor] = None, *,
+             out: Optional[Tuple[torch.Tensor, torch.Tensor, torch.Tensor]] = None,
+             stream=None) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
+    """llama_attn_qkv_rope.  x [T, hidden], w_qkv [(H+2Hkv)D, hidden] -> q [T,H,D], k, v [T,Hkv,D]."""
+    lib = load()
+    T, hidden = x.shape
+    if out is None:
+        q = torch.empty(T, n_heads, head_dim, device=x.device, dtype=x.dtype)
+        k = torch.empty(T, n_kv_heads, head_dim, device=x.device, dtype=x.dtype)
+        v = torch.empty_like(k)
+    else:
+        q, k, v = out
+    _check(lib.llama_attn_qkv_rope(_ptr(x), _ptr(w_qkv), _ptr(cos), _ptr(sin), T, hidden, n_heads,
+                                   n_kv_heads, head_dim, _ptr(q), _ptr(k), _ptr(v),
+                                   _dtype_code(x.dtype), _stream(stream)), "llama_attn_qkv_rope")
+    return q, k, v
+
+
+def out_proj(attn: torch.Tensor, w_o: torch.Tensor, *, out: Optional[torch.Tensor] = None,
+             stream=None) -> torch.Tensor:
+    """llama_attn_out_proj.  attn [T, in], w_o [out, in] -> y [T, out]."""
+    lib = load()
+    attn2 = attn.reshape(attn.shape[0], -1)
+    T, d_in = attn2.shape
+    d_out = w_o.shape[0]
+    if out is None:
+        out = torch.empty(T, d_out, device=attn.device, dtype=attn.dtype)
+    _check(lib.llama_attn_out_proj(_ptr(attn2), _ptr(w_o), T, d_in, d_out, _ptr(out),
+                                   _dtype_code(attn.dtype), _stream(stream)), "llama_attn_out_proj")
+    return out
 
 
 def prefill_workspace_bytes(bsz, n_heads, n_kv_heads, seq, head_dim, dtype, has_rope) -> int:

@@ -14,6 +14,7 @@
 #include "common.cuh"
 #include "attn_fp32.cuh"
 #include "decode_bf16.cuh"
+#include "gemm_sm100.cuh"
 #include "prefill_sm100.cuh"
 #include "rope.cuh"
 
@@ -214,6 +215,29 @@ int sm_count() {
 
 static_assert(sizeof(la::DecSmem<128>) + 1024 <= 227 * 1024, "decode shared memory exceeds 227 KB");
 static_assert(sizeof(la::PfSmem<128>) + 1024 <= 227 * 1024, "prefill shared memory exceeds 227 KB");
+static_assert(sizeof(la::GmSmem) + 1024 <= 227 * 1024, "projection GEMM shared memory exceeds 227 KB");
+
+// Y = X W^T on tcgen05 (plain) or the q/k/v heads with RoPE (qkv, D = 64 / 128).
+template <bool QKV, int D>
+int gemm_bf16(const void* x, const void* w, int M, int N, int K, la::GemmParams p,
+              cudaStream_t st) {
+  CUtensorMap ta, tb;
+  const cuuint64_t adims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(M)};
+  const cuuint64_t astr[1] = {static_cast<cuuint64_t>(K) * 2};
+  const cuuint32_t abox[2] = {static_cast<cuuint32_t>(la::gm::BK), static_cast<cuuint32_t>(la::gm::BM)};
+  const cuuint64_t bdims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(N)};
+  const cuuint32_t bbox[2] = {static_cast<cuuint32_t>(la::gm::BK), static_cast<cuuint32_t>(la::gm::BN)};
+  if (!make_map(&ta, x, 2, adims, astr, abox)) return LLAMA_ERR_CUDA;
+  if (!make_map(&tb, w, 2, bdims, astr, bbox)) return LLAMA_ERR_CUDA;
+  p.M = M;
+  p.N = N;
+  p.K = K;
+  const size_t smem = sizeof(la::GmSmem) + 1024;
+  if (!ensure_smem_attr<la::gemm_bf16_kernel<QKV, D>>(smem)) return LLAMA_ERR_CUDA;
+  const dim3 grid((M + la::gm::BM - 1) / la::gm::BM, (N + la::gm::BN - 1) / la::gm::BN);
+  la::gemm_bf16_kernel<QKV, D><<<grid, la::gm::THREADS, smem, st>>>(ta, tb, p);
+  return launch_status();
+}
 
 template <int D>
 int decode_bf16(const void* q, const void* kc, const void* vc, const int* lens, const float* cos,
@@ -357,6 +381,45 @@ int llama_rope_table_ntk(const long long* pos, int bsz, int seq, int head_dim, d
   const double base = theta * std::pow(alpha, static_cast<double>(head_dim) / (head_dim - 2));
   if (!std::isfinite(base)) return LLAMA_ERR_INVALID_ARG;
   return llama_rope_table(pos, bsz, seq, head_dim, base, 1.0, cos, sin, cuda_stream);
+}
+
+int llama_attn_qkv_rope(const void* x, const void* w_qkv, const float* cos, const float* sin,
+                        int tokens, int hidden, int n_heads, int n_kv_heads, int head_dim,
+                        void* q, void* k, void* v, int dtype, void* cuda_stream) {
+  if (!x || !w_qkv || !q || !k || !v) return LLAMA_ERR_INVALID_ARG;
+  if (tokens < 1 || hidden < 1 || (hidden % 8)) return LLAMA_ERR_INVALID_ARG;
+  if (int e = check_common(1, n_heads, n_kv_heads, head_dim, dtype, cos, sin, 1.0f)) return e;
+  if (!aligned16(x) || !aligned16(w_qkv) || !aligned16(q) || !aligned16(k) || !aligned16(v) ||
+      !aligned16(cos) || !aligned16(sin))
+    return LLAMA_ERR_INVALID_ARG;
+  if (dtype != LLAMA_DT_BF16) return LLAMA_ERR_UNSUPPORTED;
+  const long long n_out = static_cast<long long>(n_heads + 2 * n_kv_heads) * head_dim;
+  if (n_out > 0x7fffffffLL) return LLAMA_ERR_INVALID_ARG;
+  la::GemmParams p{};
+  p.q = static_cast<__nv_bfloat16*>(q);
+  p.k = static_cast<__nv_bfloat16*>(k);
+  p.v = static_cast<__nv_bfloat16*>(v);
+  p.cos = cos;
+  p.sin = sin;
+  p.H = n_heads;
+  p.Hkv = n_kv_heads;
+  cudaStream_t st = as_stream(cuda_stream);
+  if (head_dim == 128)
+    return gemm_bf16<true, 128>(x, w_qkv, tokens, static_cast<int>(n_out), hidden, p, st);
+  return gemm_bf16<true, 64>(x, w_qkv, tokens, static_cast<int>(n_out), hidden, p, st);
+}
+
+int llama_attn_out_proj(const void* attn, const void* w_o, int tokens, int in_dim, int out_dim,
+                        void* y, int dtype, void* cuda_stream) {
+  if (!attn || !w_o || !y) return LLAMA_ERR_INVALID_ARG;
+  if (tokens < 1 || in_dim < 1 || out_dim < 1 || (in_dim % 8) || (out_dim % 8))
+    return LLAMA_ERR_INVALID_ARG;
+  if (dtype != LLAMA_DT_BF16 && dtype != LLAMA_DT_F32) return LLAMA_ERR_INVALID_ARG;
+  if (!aligned16(attn) || !aligned16(w_o) || !aligned16(y)) return LLAMA_ERR_INVALID_ARG;
+  if (dtype != LLAMA_DT_BF16) return LLAMA_ERR_UNSUPPORTED;
+  la::GemmParams p{};
+  p.y = static_cast<__nv_bfloat16*>(y);
+  return gemm_bf16<false, 128>(attn, w_o, tokens, out_dim, in_dim, p, as_stream(cuda_stream));
 }
 
 size_t llama_attn_prefill_workspace_bytes(int bsz, int n_heads, int n_kv_heads, int seq,

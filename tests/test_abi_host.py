@@ -210,6 +210,36 @@ def test_rope_table_ntk_rejects(lib, args):
     assert lib.llama_rope_table_ntk(*args, None) == 1
 
 
+def _qkv(lib, **kw):
+    a = dict(x=FAKE, w=FAKE, cos=None, sin=None, T=10, hidden=64, H=8, Hkv=2, D=128, q=FAKE, k=FAKE,
+             v=FAKE, dtype=1, stream=None)
+    a.update(kw)
+    return lib.llama_attn_qkv_rope(a["x"], a["w"], a["cos"], a["sin"], a["T"], a["hidden"], a["H"],
+                                   a["Hkv"], a["D"], a["q"], a["k"], a["v"], a["dtype"], a["stream"])
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(x=None), 1), (dict(w=None), 1), (dict(v=None), 1),
+    (dict(T=0), 1), (dict(hidden=0), 1), (dict(hidden=60), 1),
+    (dict(H=8, Hkv=3), 1), (dict(cos=FAKE), 1), (dict(q=FAKE + 2), 1),
+    (dict(dtype=0), 2), (dict(D=96), 2),
+])
+def test_qkv_rope_rejects(lib, kw, status):
+    assert _qkv(lib, **kw) == status
+
+
+@pytest.mark.parametrize("args,status", [
+    ((None, FAKE, 10, 64, 64, FAKE, 1, None), 1),
+    ((FAKE, FAKE, 0, 64, 64, FAKE, 1, None), 1),
+    ((FAKE, FAKE, 10, 60, 64, FAKE, 1, None), 1),
+    ((FAKE, FAKE, 10, 64, 65, FAKE, 1, None), 1),
+    ((FAKE, FAKE, 10, 64, 64, FAKE + 4, 1, None), 1),
+    ((FAKE, FAKE, 10, 64, 64, FAKE, 0, None), 2),
+])
+def test_out_proj_rejects(lib, args, status):
+    assert lib.llama_attn_out_proj(*args) == status
+
+
 def _decode_append(lib, **kw):
     a = dict(q=FAKE, kn=FAKE, vn=FAKE, kc=FAKE, vc=FAKE, lens=FAKE, cos=None, sin=None, bsz=2, H=8,
              Hkv=2, L=100, D=128, scale=0.1, out=FAKE, ws=FAKE, ws_bytes=1 << 30, dtype=1,
