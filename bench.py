@@ -619,7 +619,6 @@ def run_configs(args):
                               "value": round(tflops, 2), "unit": "TFLOP/s",
                               "frac": round(tflops / peak_burst, 4),
                               "peak": f"{peak_burst} TFLOP/s ({peak_src} bf16 burst)"}), flush=True)
-        del q, k, v, out, wsp, x
         if cfg.name == "llama70b":
             # the NTK-aware scaled RoPE table for the workload's positions (alpha 4)
             # a small kernel: replay the captured call, so that the binding's
@@ -687,6 +686,8 @@ def run_configs(args):
                               "unit": "TFLOP/s", "frac": round(tf / peak_burst, 4),
                               "peak": f"{peak_burst} TFLOP/s ({peak_src} bf16 burst)"}), flush=True)
             del px, pw, pwo, bufs, py
+        del q, k, v, out, wsp, x
+
     for cfg in W.DECODE_CONFIGS.values():
         if not wanted(cfg):
             continue
