@@ -30,6 +30,10 @@ constexpr int STAGES = 4;
 constexpr int THREADS = 192;
 constexpr uint32_t A_BYTES = BM * BK * 2;  // 16 KB
 constexpr uint32_t B_BYTES = BN * BK * 2;  // 32 KB
+// Tiles are taken in groups of GROUP_M row tiles that sweep every column tile
+// before the next group starts: a group's rows of X (16 x 128 rows) stay in L2
+// while W streams past, so X is read from DRAM about once and W once per group.
+constexpr int GROUP_M = 16;
 }  // namespace gm
 
 struct GemmParams {
@@ -72,7 +76,12 @@ __global__ void __launch_bounds__(gm::THREADS, 1)
   GmSmem& s = *reinterpret_cast<GmSmem*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int m0 = blockIdx.x * BM, n0 = blockIdx.y * BN;
+  const int n_m = (p.M + BM - 1) / BM, n_n = (p.N + BN - 1) / BN;
+  const int group = blockIdx.x / (GROUP_M * n_n);
+  const int first_m = group * GROUP_M;
+  const int gsize = min(GROUP_M, n_m - first_m);
+  const int local = blockIdx.x - group * GROUP_M * n_n;
+  const int m0 = (first_m + local % gsize) * BM, n0 = (local / gsize) * BN;
   const int nk = (p.K + BK - 1) / BK;
 
   if (threadIdx.x == 0) {

@@ -234,8 +234,10 @@ int gemm_bf16(const void* x, const void* w, int M, int N, int K, la::GemmParams 
   p.K = K;
   const size_t smem = sizeof(la::GmSmem) + 1024;
   if (!ensure_smem_attr<la::gemm_bf16_kernel<QKV, D>>(smem)) return LLAMA_ERR_CUDA;
-  const dim3 grid((M + la::gm::BM - 1) / la::gm::BM, (N + la::gm::BN - 1) / la::gm::BN);
-  la::gemm_bf16_kernel<QKV, D><<<grid, la::gm::THREADS, smem, st>>>(ta, tb, p);
+  const long long tiles = static_cast<long long>((M + la::gm::BM - 1) / la::gm::BM) *
+                          ((N + la::gm::BN - 1) / la::gm::BN);
+  if (tiles > 0x7fffffffLL) return LLAMA_ERR_INVALID_ARG;
+  la::gemm_bf16_kernel<QKV, D><<<static_cast<unsigned>(tiles), la::gm::THREADS, smem, st>>>(ta, tb, p);
   return launch_status();
 }
 
