@@ -16,6 +16,9 @@
 // operands are 4 KB of X and 8 KB of W per 128 cycles, inside what the tensor
 // core reads from shared memory per cycle), K in blocks of 64 (one 128-byte
 // swizzle row) through a 4-stage TMA ring.
+// Persistent: one CTA per SM walks tiles blockIdx.x, + gridDim.x, ...  The
+// accumulator is double-buffered in TMEM (2 x 256 columns, all of it), so the
+// epilogue of one tile runs while the MMAs of the next fill the other buffer.
 // Warps: 0 TMA producer, 1 TMEM allocator + MMA issuer, 2-5 epilogue (one
 // output row per thread; warp w reaches TMEM lanes of quarter w % 4).
 #pragma once
@@ -51,7 +54,9 @@ struct GmSmem {
   alignas(1024) __nv_bfloat16 a[gm::STAGES][gm::BM * gm::BK];
   alignas(1024) __nv_bfloat16 b[gm::STAGES][gm::BN * gm::BK];
   uint64_t full[gm::STAGES], empty[gm::STAGES];
-  uint64_t acc_full;
+  uint64_t acc_full[2];   // accumulator buffer holds a finished tile (MMA commit)
+  uint64_t acc_empty[2];  // its epilogue has read it (one arrive per epilogue warp)
+  uint64_t mma_done;      // every MMA this CTA issued has completed
   uint32_t tmem_base;
 };
 
@@ -70,26 +75,35 @@ __global__ void __launch_bounds__(gm::THREADS, 1)
     gemm_bf16_kernel(const __grid_constant__ CUtensorMap tm_a,
                      const __grid_constant__ CUtensorMap tm_b, GemmParams p) {
   using namespace gm;
-  constexpr uint32_t TMEM_COLS = BN;
+  constexpr uint32_t TMEM_COLS = 2 * BN;
   constexpr uint32_t IDESC = idesc_bf16(BM, BN, false);
   extern __shared__ uint8_t smem_raw[];
   GmSmem& s = *reinterpret_cast<GmSmem*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_m = (p.M + BM - 1) / BM, n_n = (p.N + BN - 1) / BN;
-  const int group = blockIdx.x / (GROUP_M * n_n);
-  const int first_m = group * GROUP_M;
-  const int gsize = min(GROUP_M, n_m - first_m);
-  const int local = blockIdx.x - group * GROUP_M * n_n;
-  const int m0 = (first_m + local % gsize) * BM, n0 = (local / gsize) * BN;
+  const int n_tiles = n_m * n_n;
   const int nk = (p.K + BK - 1) / BK;
+  // tile index -> (first row, first column)
+  auto tile_origin = [&](int tile, int& m0, int& n0) {
+    const int group = tile / (GROUP_M * n_n);
+    const int first_m = group * GROUP_M;
+    const int gsize = min(GROUP_M, n_m - first_m);
+    const int local = tile - group * GROUP_M * n_n;
+    m0 = (first_m + local % gsize) * BM;
+    n0 = (local / gsize) * BN;
+  };
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < STAGES; ++i) {
       mbar_init(&s.full[i], 1);
       mbar_init(&s.empty[i], 1);
     }
-    mbar_init(&s.acc_full, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&s.acc_full[i], 1);
+      mbar_init(&s.acc_empty[i], 4);
+    }
+    mbar_init(&s.mma_done, 1);
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -108,60 +122,86 @@ __global__ void __launch_bounds__(gm::THREADS, 1)
       tma_prefetch_desc(&tm_b);
     }
     __syncwarp();
-    int issued = 0;
-    for (int kb = 0; kb < nk; ++kb) {
-      const int st = kb % STAGES;
-      if (kb >= STAGES && !mbar_wait(&s.empty[st], ((kb / STAGES) - 1) & 1)) break;
-      if (elect_one()) {
-        mbar_arrive_expect_tx(&s.full[st], A_BYTES + B_BYTES);
-        tma_load_2d(&s.a[st][0], &tm_a, &s.full[st], kb * BK, m0);
-        tma_load_2d(&s.b[st][0], &tm_b, &s.full[st], kb * BK, n0);
+    int it = 0;  // k-blocks issued by this CTA, over all its tiles
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x) {
+      int m0, n0;
+      tile_origin(tile, m0, n0);
+      for (int kb = 0; kb < nk; ++kb, ++it) {
+        const int st = it % STAGES;
+        if (it >= STAGES && !mbar_wait(&s.empty[st], ((it / STAGES) - 1) & 1)) {
+          ok = false;
+          break;
+        }
+        if (elect_one()) {
+          mbar_arrive_expect_tx(&s.full[st], A_BYTES + B_BYTES);
+          tma_load_2d(&s.a[st][0], &tm_a, &s.full[st], kb * BK, m0);
+          tma_load_2d(&s.b[st][0], &tm_b, &s.full[st], kb * BK, n0);
+        }
+        __syncwarp();
       }
-      __syncwarp();
-      issued = kb + 1;
     }
     // leave no copy in flight
-    for (int kb = max(0, issued - STAGES); kb < issued; ++kb)
-      if (!mbar_wait(&s.full[kb % STAGES], (kb / STAGES) & 1)) break;
+    for (int i = max(0, it - STAGES); i < it; ++i)
+      if (!mbar_wait(&s.full[i % STAGES], (i / STAGES) & 1)) break;
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     const uint64_t a_desc0 = sw128_desc(smem_u32(&s.a[0][0]), 16, 1024);
     const uint64_t b_desc0 = sw128_desc(smem_u32(&s.b[0][0]), 16, 1024);
     bool ok = true;
-    for (int kb = 0; kb < nk && ok; ++kb) {
-      const int st = kb % STAGES;
-      ok = mbar_wait(&s.full[st], (kb / STAGES) & 1);
-      if (!ok) break;
+    int it = 0;  // k-blocks consumed, over all tiles
+    int i = 0;   // tiles of this CTA
+    for (int tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x, ++i) {
+      const int acc = i & 1;
+      // the epilogue has read this buffer's previous tile (i - 2)
+      if (i >= 2 && !mbar_wait(&s.acc_empty[acc], ((i >> 1) - 1) & 1)) break;
       tc_fence_after();
-      if (elect_one()) {
+      const uint32_t d_tmem = tmem + static_cast<uint32_t>(acc * BN);
+      for (int kb = 0; kb < nk; ++kb, ++it) {
+        const int st = it % STAGES;
+        ok = mbar_wait(&s.full[st], (it / STAGES) & 1);
+        if (!ok) break;
+        tc_fence_after();
+        if (elect_one()) {
 #pragma unroll
-        for (int kk = 0; kk < BK / 16; ++kk) {
-          const uint64_t ad = a_desc0 + ((static_cast<uint32_t>(st) * A_BYTES + kk * 32) >> 4);
-          const uint64_t bd = b_desc0 + ((static_cast<uint32_t>(st) * B_BYTES + kk * 32) >> 4);
-          mma_ss(tmem, ad, bd, IDESC, (kb > 0 || kk > 0) ? 1u : 0u);
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            const uint64_t ad = a_desc0 + ((static_cast<uint32_t>(st) * A_BYTES + kk * 32) >> 4);
+            const uint64_t bd = b_desc0 + ((static_cast<uint32_t>(st) * B_BYTES + kk * 32) >> 4);
+            mma_ss(d_tmem, ad, bd, IDESC, (kb > 0 || kk > 0) ? 1u : 0u);
+          }
+          tc_commit(&s.empty[st]);
         }
-        tc_commit(&s.empty[st]);
+        __syncwarp();
       }
+      if (!ok) break;
+      if (elect_one()) tc_commit(&s.acc_full[acc]);  // the tile's MMAs have completed when it fires
       __syncwarp();
     }
-    if (elect_one()) tc_commit(&s.acc_full);  // every MMA above has completed when it fires
+    // no MMA may still run when the TMEM is released
+    if (elect_one()) tc_commit(&s.mma_done);
     __syncwarp();
-    mbar_wait(&s.acc_full, 0);
+    mbar_wait(&s.mma_done, 0);
   } else {
     // ------------------------------------------------------------ epilogue
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;
-    const int m = m0 + r;  // output row (token)
-    const bool row_ok = m < p.M;
-    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
-    if (mbar_wait(&s.acc_full, 0)) {
+    int i = 0;
+    for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++i) {
+      const int acc = i & 1;
+      int m0, n0;
+      tile_origin(tile, m0, n0);
+      const int m = m0 + r;  // output row (token)
+      const bool row_ok = m < p.M;
+      if (!mbar_wait(&s.acc_full[acc], (i >> 1) & 1)) break;
       tc_fence_after();
+      const uint32_t t_acc = tmem + static_cast<uint32_t>(acc * BN) +
+                             (static_cast<uint32_t>(quarter * 32) << 16);
       if constexpr (!QKV) {
 #pragma unroll 1
         for (int c = 0; c < BN / 32; ++c) {
-          uint32_t acc[32];
-          tmem_ld32(tmem + lane_off + c * 32, acc);
-          tmem_ld_wait(acc);
+          uint32_t acc_r[32];
+          tmem_ld32(t_acc + c * 32, acc_r);
+          tmem_ld_wait(acc_r);
           const int n = n0 + c * 32;
           if (row_ok && n < p.N) {
             __nv_bfloat16* dst = p.y + static_cast<size_t>(m) * p.N + n;
@@ -169,10 +209,10 @@ __global__ void __launch_bounds__(gm::THREADS, 1)
             for (int e = 0; e < 32; e += 8) {
               if (n + e + 8 <= p.N) {
                 uint4 w;
-                w.x = pack_bf16x2(__uint_as_float(acc[e]), __uint_as_float(acc[e + 1]));
-                w.y = pack_bf16x2(__uint_as_float(acc[e + 2]), __uint_as_float(acc[e + 3]));
-                w.z = pack_bf16x2(__uint_as_float(acc[e + 4]), __uint_as_float(acc[e + 5]));
-                w.w = pack_bf16x2(__uint_as_float(acc[e + 6]), __uint_as_float(acc[e + 7]));
+                w.x = pack_bf16x2(__uint_as_float(acc_r[e]), __uint_as_float(acc_r[e + 1]));
+                w.y = pack_bf16x2(__uint_as_float(acc_r[e + 2]), __uint_as_float(acc_r[e + 3]));
+                w.z = pack_bf16x2(__uint_as_float(acc_r[e + 4]), __uint_as_float(acc_r[e + 5]));
+                w.w = pack_bf16x2(__uint_as_float(acc_r[e + 6]), __uint_as_float(acc_r[e + 7]));
                 *reinterpret_cast<uint4*>(dst + e) = w;
               }
             }
@@ -202,8 +242,8 @@ __global__ void __launch_bounds__(gm::THREADS, 1)
           for (int j = 0; j < D / 64; ++j) {
             // columns d in [32j, 32j + 32) and their rotation partners d + D/2
             uint32_t x1[32], x2[32];
-            tmem_ld32(tmem + lane_off + hl * D + 32 * j, x1);
-            tmem_ld32(tmem + lane_off + hl * D + D / 2 + 32 * j, x2);
+            tmem_ld32(t_acc + hl * D + 32 * j, x1);
+            tmem_ld32(t_acc + hl * D + D / 2 + 32 * j, x2);
             tmem_ld_wait(x1);
             tmem_ld_wait(x2);
 #pragma unroll
@@ -252,6 +292,11 @@ __global__ void __launch_bounds__(gm::THREADS, 1)
           }
         }
       }
+      // every tcgen05.ld of this buffer has completed (waited above): hand it
+      // back to the MMA warp for tile i + 2
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s.acc_empty[acc]);
     }
   }
 

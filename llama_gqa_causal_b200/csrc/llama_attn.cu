@@ -237,7 +237,11 @@ int gemm_bf16(const void* x, const void* w, int M, int N, int K, la::GemmParams 
   const long long tiles = static_cast<long long>((M + la::gm::BM - 1) / la::gm::BM) *
                           ((N + la::gm::BN - 1) / la::gm::BN);
   if (tiles > 0x7fffffffLL) return LLAMA_ERR_INVALID_ARG;
-  la::gemm_bf16_kernel<QKV, D><<<static_cast<unsigned>(tiles), la::gm::THREADS, smem, st>>>(ta, tb, p);
+  const int sms = sm_count();
+  if (sms <= 0) return LLAMA_ERR_CUDA;
+  // persistent: one CTA per SM (198 KB of shared memory each), tiles strided by the grid
+  const unsigned grid = static_cast<unsigned>(std::min<long long>(tiles, sms));
+  la::gemm_bf16_kernel<QKV, D><<<grid, la::gm::THREADS, smem, st>>>(ta, tb, p);
   return launch_status();
 }
 

@@ -37,6 +37,10 @@ def _weights(n_out, n_in, g):
 QKV_CASES = [
     # (tokens, hidden, H, Hkv, D, rope)
     (200, 512, 8, 2, 128, True),    # ragged token count (two M tiles, the second partial)
+    # 20 x 24 = 480 tiles: every CTA of the persistent grid takes three or four,
+    # so both TMEM accumulator buffers are reused; 20 row tiles = one group of
+    # 16 and a short group of 4, the last row tile ragged
+    (2500, 256, 32, 8, 128, True),
     (130, 256, 4, 4, 64, True),     # head_dim 64: four heads per 256-column tile
     (1, 128, 8, 1, 128, True),      # one token, MQA
     (300, 1000, 4, 2, 128, False),  # no RoPE; hidden not a multiple of the 64-wide K block
@@ -77,7 +81,8 @@ def test_qkv_rope_matches_oracle(case):
     _close(v, ev, f"{case} v")
 
 
-@pytest.mark.parametrize("T,d_in,d_out", [(200, 512, 520), (1, 64, 256), (257, 1000, 768)])
+@pytest.mark.parametrize("T,d_in,d_out", [(200, 512, 520), (1, 64, 256), (257, 1000, 768),
+                                          (3000, 384, 4096)])  # 24 x 16 tiles
 def test_out_proj_matches_oracle(T, d_in, d_out):
     g = torch.Generator().manual_seed(T + d_in + d_out)
     a = W.normal((T, d_in), torch.bfloat16, g)
@@ -111,4 +116,28 @@ def test_attention_block_matches_oracle_chain():
     ref_y = ref_attn @ w_o.double().numpy().T
     err = _close(y, ref_y, "attention block")
     PARITY_REPORT.append(("attention block (qkv+rope, prefill, o_proj)", "bfloat16",
+                          float(err.max()), float(err.mean())))
+
+
+def test_qkv_rope_70b_shape_sampled_rows():
+    # the 70B projection at full size (8192 tokens, hidden 8192, 64 + 2 x 8 heads
+    # of 128), the launch the projection benchmark times; rows sampled from every
+    # group of row tiles and the last tile, all columns checked
+    T, hidden, H, Hkv, D = 8192, 8192, 64, 8, 128
+    g = torch.Generator().manual_seed(70)
+    x = W.normal((T, hidden), torch.bfloat16, g)
+    w = _weights((H + 2 * Hkv) * D, hidden, g)
+    pos = torch.arange(T)
+    dev = torch.device("cuda")
+    cos, sin = api.rope_table(pos.view(1, -1).to(dev), D, THETA, 1.0)
+    q, k, v = api.qkv_rope(x.to(dev), w.to(dev), H, Hkv, D, cos.view(T, D), sin.view(T, D))
+    torch.cuda.synchronize()
+    assert api.device_status() == api.LLAMA_OK
+    rows = torch.tensor(sorted({0, 1, 127, 128, 2047, 2048, 4095, 4096, 6143, 6144, 8190, 8191}
+                               | set(torch.randint(0, T, (20,), generator=g).tolist())))
+    eq, ek, ev = _qkv_expected(x[rows], w, pos[rows], H, Hkv, D, True)
+    errs = [_close(q.cpu()[rows], eq, "q"), _close(k.cpu()[rows], ek, "k"),
+            _close(v.cpu()[rows], ev, "v")]
+    err = np.concatenate([e.reshape(-1) for e in errs])
+    PARITY_REPORT.append(("qkv+rope projection 70B shape (sampled rows)", "bfloat16",
                           float(err.max()), float(err.mean())))
