@@ -223,6 +223,8 @@ DECODE_CASES = [
     (300, 8, 8, 64, 96, None),              # prefix runs of several batch entries per thread
     (3, 8, 2, 128, 200, [0, 0, 0]),          # no work at all: zero output everywhere
     (4, 16, 2, 128, 300, [-3, 301, 1000, 150]),  # lengths outside [0, L] are clamped
+    (4096, 8, 1, 64, 64, None),             # the largest batch the bf16 decode takes
+    (2, 8, 1, 128, 32768, [32768, 20001]),  # long caches: shares of hundreds of chunks
 ]
 
 
@@ -248,6 +250,18 @@ def test_decode_small(case, dtype):
     for i, n in enumerate(clamped):
         if n == 0:
             assert torch.all(out[i].float().cpu() == 0)
+
+
+def test_prefill_long_sequence_sampled_rows():
+    # S = 16384: the (batch, K/V head) pairs whose K/V fit in L2 run as bundles
+    # of several pairs, and the last position blocks stream 128 K/V tiles
+    cfg, x = W.small_prefill(2, 16384, 16, 2, 128, torch.bfloat16, causal=True, seed=43)
+    out = _gpu_prefill(cfg, x)
+    ref = np.full(out.shape, np.nan)
+    for lo, hi in [(0, 64), (8160, 8224), (16320, 16384)]:
+        part = _oracle_prefill(cfg, x, rows=(lo, hi))
+        ref[:, lo:hi] = part[:, lo:hi]
+    _check(out, ref, torch.bfloat16, "S 16384 (sampled rows)", report=True)
 
 
 def test_decode_equals_last_prefill_row_on_gpu():
