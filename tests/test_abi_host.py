@@ -9,6 +9,7 @@ import os
 import re
 
 import pytest
+import torch
 
 from llama_gqa_causal_b200 import api, build
 
@@ -308,5 +309,17 @@ def test_loader_refuses_a_library_built_from_other_sources(lib, monkeypatch):
     monkeypatch.setattr(build, "built_hash", lambda: "0" * 64)
     with pytest.raises(RuntimeError, match="other sources"):
         api.load()
+    monkeypatch.undo()
+    assert api.load() is not None
+
+
+def test_loader_fails_loudly_without_the_library(tmp_path, monkeypatch):
+    # No CPU fallback: without the built library every entry point raises.
+    monkeypatch.setattr(api, "_lib", None)
+    monkeypatch.setattr(api, "LIB_PATH", str(tmp_path / "libllama_attn.so"))
+    with pytest.raises(RuntimeError, match="is missing"):
+        api.load()
+    with pytest.raises(RuntimeError, match="is missing"):
+        api.rope_table(torch.zeros(1, 4, dtype=torch.int64), 128)
     monkeypatch.undo()
     assert api.load() is not None
