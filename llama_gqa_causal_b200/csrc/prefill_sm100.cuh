@@ -72,6 +72,12 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 units
 #define LA_POLY_PAIRS_OF_8 3
 #endif
 constexpr int kPolyPairsOf8 = LA_POLY_PAIRS_OF_8;
+// Pairs of the second P half exponentiated before the wait for the first
+// half's TMEM store.
+#ifndef LA_PF_ST_OVERLAP
+#define LA_PF_ST_OVERLAP 8
+#endif
+constexpr int kStOverlap = LA_PF_ST_OVERLAP;
 }  // namespace pf
 
 struct PrefillParams {
@@ -547,12 +553,13 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
           const float cc = kEdge ? 1.f : c_log2;
           float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
           // P in two halves (keys 0-63, 64-127): the MMA warp starts O += P V on the
-          // first half while the second is being exponentiated
+          // first half while the second is being exponentiated.  The first
+          // kStOverlap pairs of the second half are computed between the first
+          // half's TMEM store and the wait for it, which hides the store's latency.
+          uint32_t pk[2][32];
+          auto exps = [&](int e0, int e1) {  // pairs of keys [e0, e1)
 #pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            uint32_t pk[32];
-#pragma unroll
-            for (int e = h * 64; e < h * 64 + 64; e += 2) {
+            for (int e = e0; e < e1; e += 2) {
               float a0, a1, p0, p1;
               ffma2(a0, a1, v[e], v[e + 1], cc, cc, nref, nref);  // exponent = v*c - m_ref
               if (!kEdge && ((e / 2) % 8) < kPolyPairsOf8) {
@@ -563,28 +570,36 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
               }
               const int k = (e / 2) % 4;
               fadd2(acc[2 * k], acc[2 * k + 1], acc[2 * k], acc[2 * k + 1], p0, p1);
-              pk[(e % 64) / 2] = pack_bf16x2(p0, p1);
+              pk[e / 64][(e % 64) / 2] = pack_bf16x2(p0, p1);
             }
-            if (h == 0 && jj > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
-              // O correction before any P of this tile is released (warp-collective
-              // TMEM access when any row of the warp needs it); PV_{j-1} has
-              // completed: its commit preceded this tile's S
-#pragma unroll
-              for (int c = 0; c < D / 32; ++c) {
-                uint32_t orr[32];
-                tmem_ld32(my_o + lane_off + c * 32, orr);
-                tmem_ld_wait(orr);
-#pragma unroll
-                for (int e = 0; e < 32; ++e) orr[e] = __float_as_uint(__uint_as_float(orr[e]) * alpha);
-                tmem_st32(my_o + lane_off + c * 32, orr);
-              }
-            }
-            tmem_st32(my_s + lane_off + h * 32, pk);
+          };
+          auto release = [&](uint64_t* bar) {
             tmem_st_wait();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(h == 0 ? &s.p_lo[t] : &s.p_hi[t]);
+            if (lane == 0) mbar_arrive(bar);
+          };
+          exps(0, 64);
+          if (jj > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+            // O correction before any P of this tile is released (warp-collective
+            // TMEM access when any row of the warp needs it); PV_{j-1} has
+            // completed: its commit preceded this tile's S
+#pragma unroll
+            for (int c = 0; c < D / 32; ++c) {
+              uint32_t orr[32];
+              tmem_ld32(my_o + lane_off + c * 32, orr);
+              tmem_ld_wait(orr);
+#pragma unroll
+              for (int e = 0; e < 32; ++e) orr[e] = __float_as_uint(__uint_as_float(orr[e]) * alpha);
+              tmem_st32(my_o + lane_off + c * 32, orr);
+            }
           }
+          tmem_st32(my_s + lane_off, pk[0]);
+          exps(64, 64 + 2 * kStOverlap);
+          release(&s.p_lo[t]);
+          exps(64 + 2 * kStOverlap, 128);
+          tmem_st32(my_s + lane_off + 32, pk[1]);
+          release(&s.p_hi[t]);
           rs = ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
           l_sum = fmaf(l_sum, alpha, rs);
         };
