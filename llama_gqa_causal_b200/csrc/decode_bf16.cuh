@@ -167,6 +167,11 @@ __global__ void __launch_bounds__(dec::THREADS, 1) decode_bf16_kernel(
     tma_prefetch_desc(&tm_k);
     tma_prefetch_desc(&tm_v);
   }
+  // Launched as a programmatic dependent of whatever precedes it on the stream:
+  // the CTAs may be resident before that grid has finished, so nothing in
+  // global memory is read or written before this wait (the previous decode's
+  // combine still reads the workspace this kernel writes).
+  asm volatile("griddepcontrol.wait;" ::: "memory");
 
   // ---- chunk counts per batch entry, prefix-summed (identical in every CTA):
   // each thread sums a contiguous run of entries, the run totals are scanned
@@ -526,6 +531,9 @@ __global__ void __launch_bounds__(dec::COMBINE_THREADS) decode_combine_kernel(
   const int seq = blockIdx.x, b = blockIdx.y;
   const int kvh = seq / hchunks, hc = seq - kvh * hchunks;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  // a programmatic dependent launched after this kernel (the next decode) may
+  // be scheduled now; it waits for this grid to finish before touching memory
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   // chunks of batch entries < b and of all entries: block-wide sums over lens
   __shared__ long long red[2][NW];
   long long before = 0, all = 0;

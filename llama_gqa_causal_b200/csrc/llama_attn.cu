@@ -281,24 +281,37 @@ int decode_bf16(const void* q, const void* kc, const void* vc, const int* lens, 
   p.scale_log2 = scale * 1.4426950408889634f;
   const size_t smem = sizeof(la::DecSmem<D>) + 1024;
   const int append = (k_new != nullptr) ? 1 : 0;
+  // Both kernels launch as programmatic dependents of what precedes them on
+  // the stream: their blocks are scheduled while the previous grid drains and
+  // wait on the device (griddepcontrol.wait) before touching global memory.
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t scfg = {};
+  scfg.gridDim = dim3(n_ctas);
+  scfg.blockDim = dim3(la::dec::THREADS);
+  scfg.dynamicSmemBytes = smem;
+  scfg.stream = st;
+  scfg.attrs = attr;
+  scfg.numAttrs = 1;
+  cudaError_t se;
   if (append) {
     if (!ensure_smem_attr<la::decode_bf16_kernel<D, true>>(smem)) return LLAMA_ERR_CUDA;
-    la::decode_bf16_kernel<D, true><<<n_ctas, la::dec::THREADS, smem, st>>>(tk, tv, p);
+    se = cudaLaunchKernelEx(&scfg, la::decode_bf16_kernel<D, true>, tk, tv, p);
   } else {
     if (!ensure_smem_attr<la::decode_bf16_kernel<D, false>>(smem)) return LLAMA_ERR_CUDA;
-    la::decode_bf16_kernel<D, false><<<n_ctas, la::dec::THREADS, smem, st>>>(tk, tv, p);
+    se = cudaLaunchKernelEx(&scfg, la::decode_bf16_kernel<D, false>, tk, tv, p);
+  }
+  if (se != cudaSuccess) {
+    fprintf(stderr, "llama_attn: decode launch failed: %s\n", cudaGetErrorString(se));
+    return LLAMA_ERR_CUDA;
   }
   if (int e = launch_status()) return e;
-  // the combine launches as a programmatic dependent of the split kernel: its
-  // blocks are scheduled while the split kernel drains and wait on the device
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(Hkv * p.hchunks, bsz);
   cfg.blockDim = dim3(la::dec::COMBINE_THREADS);
   cfg.dynamicSmemBytes = 0;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   const float* home = p.ws_home;

@@ -21,6 +21,9 @@ __global__ void rope_table_kernel(const long long* __restrict__ pos, long long n
                                   float* __restrict__ sin_out) {
   // blockDim.x is a multiple of D/2: each thread keeps one frequency index i
   // (so its inverse frequency is formed once) and walks the rows
+  // a programmatic dependent launched after this kernel (a decode reading the
+  // table) may be scheduled now; it waits for this grid to finish
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int half = D / 2;
   const int i = static_cast<int>(threadIdx.x % half);
   const int rows_per_block = static_cast<int>(blockDim.x / half);
