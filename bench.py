@@ -468,6 +468,41 @@ def _oracle_sample_prefill(cfg, rows):
     return dt, flops
 
 
+def _config_cpu_baseline(cfg, x):
+    """The fp64 oracle timed on a bounded sample of one named workload, on all
+    host cores and on one core; the value in the workload's own unit."""
+    import oracle
+    out = {"kind": "oracle"}
+    for key, nthreads in (("value", 0), ("one_core", 1)):
+        if isinstance(cfg, W.DecodeConfig):
+            # the whole step: every cached row attended once
+            t = time.perf_counter()
+            oracle.decode(x["q"], x["k_cache"], x["v_cache"], x["lens"], x["qpos"], theta=cfg.theta,
+                          factor=cfg.factor, scale=cfg.scale, nthreads=nthreads)
+            dt = time.perf_counter() - t
+            nbytes = 2 * int(x["lens"].to(torch.int64).sum()) * cfg.n_kv_heads * cfg.head_dim * 2
+            out[key] = round(nbytes / dt / 1e9, 4)
+            out.update(unit="GB/s", sample="the whole step (all batch entries and heads)")
+            continue
+        # prefill: all heads of the last rows (every row for the small workloads)
+        lo = 0 if cfg.seq <= 256 else cfg.seq - 64
+        reps = 20 if cfg.seq <= 64 else 1
+        t = time.perf_counter()
+        for _ in range(reps):
+            oracle.prefill(x["q"], x["k"], x["v"], x["pos"], theta=cfg.theta, factor=cfg.factor,
+                           scale=cfg.scale, causal=cfg.causal, rows=(lo, cfg.seq), nthreads=nthreads)
+        dt = (time.perf_counter() - t) / reps
+        keys = sum(min(cfg.seq, i + 1) if cfg.causal else cfg.seq for i in range(lo, cfg.seq))
+        flops = 4 * cfg.head_dim * keys * cfg.bsz * cfg.n_heads
+        out[key] = round(flops / dt / 1e12, 6)
+        out.update(unit="TFLOP/s",
+                   sample=("every row" if lo == 0 else f"query rows [{lo}, {cfg.seq})")
+                   + f" of all {cfg.n_heads} heads and {cfg.bsz} batch "
+                   + ("entry" if cfg.bsz == 1 else "entries") + f" ({flops / 1e9:.3g} GFLOP)")
+    out["cores"] = oracle.max_threads()
+    return out
+
+
 def cpu_baseline(rows=None):
     import oracle
     cfg = PREFILL
@@ -563,10 +598,13 @@ def run_configs(args):
         ms = timed(lambda: api.prefill(q, k, v, cos, sin, causal=cfg.causal, scale=cfg.scale,
                                        out=out, workspace=wsp))
         tflops = cfg.flops() / (ms * 1e-3) / 1e12
-        print(json.dumps({"phase": "configs", "workload": cfg.name, "dtype": str(cfg.dtype).split(".")[-1],
-                          "ms_per_call": round(ms, 5), "value": round(tflops, 2), "unit": "TFLOP/s",
-                          "frac": round(tflops / peak_burst, 4),
-                          "peak": f"{peak_burst} TFLOP/s ({peak_src} bf16 burst)"}), flush=True)
+        cline = {"phase": "configs", "workload": cfg.name, "dtype": str(cfg.dtype).split(".")[-1],
+                 "ms_per_call": round(ms, 5), "value": round(tflops, 2), "unit": "TFLOP/s",
+                 "frac": round(tflops / peak_burst, 4),
+                 "peak": f"{peak_burst} TFLOP/s ({peak_src} bf16 burst)"}
+        if not args.no_cpu_baseline:
+            cline["cpu_baseline"] = _config_cpu_baseline(cfg, x)
+        print(json.dumps(cline), flush=True)
         if cfg.name == "llama7b":
             # the same batch right-padded: the second entry holds about half its rows
             lens = [cfg.seq] + [cfg.seq // 2 + 37] * (cfg.bsz - 1)
@@ -702,10 +740,12 @@ def run_configs(args):
                                       scale=cfg.scale, out=out, workspace=wsp))
         nbytes = int(2 * x["lens"].to(torch.int64).sum().item() * cfg.n_kv_heads * cfg.head_dim * 2)
         gbs = nbytes / (ms * 1e-3) / 1e9
-        print(json.dumps({"phase": "configs", "workload": cfg.name, "dtype": str(cfg.dtype).split(".")[-1],
-                          "ms_per_call": round(ms, 5), "value": round(gbs, 1), "unit": "GB/s",
-                          "frac": round(gbs / hbm, 4), "peak": f"{hbm} GB/s ({peak_src} copy)"}),
-              flush=True)
+        cline = {"phase": "configs", "workload": cfg.name, "dtype": str(cfg.dtype).split(".")[-1],
+                 "ms_per_call": round(ms, 5), "value": round(gbs, 1), "unit": "GB/s",
+                 "frac": round(gbs / hbm, 4), "peak": f"{hbm} GB/s ({peak_src} copy)"}
+        if not args.no_cpu_baseline:
+            cline["cpu_baseline"] = _config_cpu_baseline(cfg, x)
+        print(json.dumps(cline), flush=True)
         # the same step with the new token's own key/value appended at row
         # p = min(len, L - 1) and attended (rows 0..p); every call rewrites the
         # same rows with the same values
