@@ -423,6 +423,48 @@ def _decode_phase(args, ws, local, dev, stream, line):
     dec_achieved = dbytes / (ms_dec_call * 1e-3) / 1e9
     assert api.device_status() == api.LLAMA_OK
 
+    # e2e: the KV caches are model state resident in HBM; every step copies its
+    # own inputs (the new token's q, the cache lengths, the query positions)
+    # from pinned host memory, runs the public API, and reads the output back.
+    # A decode step needs the previous step's output, so the steps run one
+    # after another on one stream.
+    dec_e2e = None
+    if not args.no_e2e:
+        hosts = [{n: insts[r][n].cpu().pin_memory() for n in ("q", "lens", "qpos")} for r in range(2)]
+        hout = torch.empty(dout.shape, dtype=dout.dtype).pin_memory()
+
+        def e2e_step(i):
+            d, h = insts[i % 2], hosts[i % 2]
+            for n in ("q", "lens", "qpos"):
+                d[n].copy_(h[n], non_blocking=True)
+            decode_step(i)
+            hout.copy_(dout, non_blocking=True)
+
+        for i in range(max(args.warmup, 3)):
+            e2e_step(i)
+        torch.cuda.synchronize()
+        _barrier(ws)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for i in range(dsteps):
+            e2e_step(i)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        _barrier(ws)
+        ms_e2e = _max_over_ranks(e0.elapsed_time(e1), ws)
+        assert api.device_status() == api.LLAMA_OK
+        dec_e2e = {
+            "value": round(replicas.job_throughput(dbytes, dsteps, ms_e2e, ws) / 1e9, 1),
+            "unit": "GB/s",
+            "ms_per_step": round(ms_e2e / dsteps, 4),
+            "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in hosts[0].values()),
+            "d2h_bytes_per_step": hout.numel() * hout.element_size(),
+            "steps": dsteps,
+            "launch": "one stream, steps in sequence, direct launches; caches resident",
+        }
+        del hosts, hout
+
     line["decode"] = {
         "launch": "cuda-graph replay" if graphs is not None else "direct",
         "value": round(dec_value, 1),
@@ -438,8 +480,10 @@ def _decode_phase(args, ws, local, dev, stream, line):
             "unit": "GB/s",
             "frac": round(dec_achieved / hbm, 4),
             "peak_source": f"{peak_src} copy bandwidth",
-            "traffic": None,
+            "traffic": _traffic("decode_bf16_kernel<128>"),
+            "traffic_unit": "bytes per launch of the split kernel (ncu dram read+write)",
         },
+        "e2e": dec_e2e,
     }
     if "value" not in line:  # decode-only run: the decode numbers are the line's
         line.update({"value": line["decode"]["value"], "unit": "GB/s",
