@@ -154,8 +154,9 @@ int oracle_prefill(const float* q, const float* k, const float* v,
   int kv_lo = h_lo / group, kv_hi = (h_hi - 1) / group + 1;
 
 #ifdef _OPENMP
-  if (nthreads > 0) omp_set_num_threads(nthreads);
-#pragma omp parallel for collapse(2) schedule(dynamic)
+  /* thread count for this call only (nthreads <= 0: the process default) */
+  const int nt = nthreads > 0 ? nthreads : omp_get_max_threads();
+#pragma omp parallel for collapse(2) schedule(dynamic) num_threads(nt)
 #endif
   for (int b = 0; b < bsz; ++b)
     for (int j = 0; j < S; ++j) {
@@ -173,7 +174,7 @@ int oracle_prefill(const float* q, const float* k, const float* v,
 
   const long n_rows = (long)bsz * (h_hi - h_lo) * (i_hi - i_lo);
 #ifdef _OPENMP
-#pragma omp parallel
+#pragma omp parallel num_threads(nt)
 #endif
   {
     double* scores = (double*)malloc(sizeof(double) * S);
@@ -234,8 +235,9 @@ int oracle_decode(const float* q, const float* k_cache, const float* v_cache,
     if (lens[b] < 0 || lens[b] > L) return -1;
   const int group = H / Hkv;
 #ifdef _OPENMP
-  if (nthreads > 0) omp_set_num_threads(nthreads);
-#pragma omp parallel
+  /* thread count for this call only (nthreads <= 0: the process default) */
+  const int nt = nthreads > 0 ? nthreads : omp_get_max_threads();
+#pragma omp parallel num_threads(nt)
 #endif
   {
     double* scores = (double*)malloc(sizeof(double) * L);

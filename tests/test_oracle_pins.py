@@ -461,3 +461,15 @@ def test_ntk_lowest_frequency_is_linear_interpolation(D, alpha):
     # and it is not plain interpolation elsewhere: a middle frequency moves less
     mid = D // 4
     assert np.abs(c_ntk[:, mid] - c_lin[:, mid]).max() > 1e-3
+
+
+def test_oracle_thread_count_applies_to_one_call_only():
+    # a one-core timing must not leave the process on one core for later calls
+    before = oracle.max_threads()
+    g = np.random.default_rng(5)
+    q = g.standard_normal((1, 8, 2, 64)).astype(np.float32)
+    k = g.standard_normal((1, 8, 1, 64)).astype(np.float32)
+    a = oracle.prefill(q, k, k, None, nthreads=1)
+    b = oracle.prefill(q, k, k, None)
+    assert oracle.max_threads() == before
+    assert np.array_equal(a, b)
