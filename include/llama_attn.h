@@ -37,7 +37,15 @@
  *     the caller, and must be 16-byte aligned.  The library never allocates
  *     device memory and never frees what it is given.
  *   - All work is enqueued on `cuda_stream` (a cudaStream_t; NULL = legacy
- *     default stream) and the call returns without synchronising.
+ *     default stream) and the call returns without synchronising.  Stream
+ *     order is kept: the decode kernels launch as programmatic dependents of
+ *     the preceding grid (their blocks may become resident early) but wait on
+ *     the device for it to finish before they read or write any memory.  The
+ *     decode combine and the RoPE table kernels allow their own programmatic
+ *     dependents to launch early; a caller kernel launched with the
+ *     programmatic-serialization attribute after them must wait
+ *     (griddepcontrol.wait / cudaGridDependencySynchronize) before reading
+ *     their outputs, as for any such launch.
  *   - `dtype` (llama_dtype) applies to q, k, v, the caches and out together.
  *     LLAMA_DT_BF16 runs the tensor-core kernels (tcgen05 prefill, mma decode)
  *     with fp32 accumulation and an fp32 softmax; the probabilities are
