@@ -21,6 +21,12 @@ from a second pass with CUDA events around each library call.
   llama_attn_decode (split-KV kernel + combine).  Bytes = K and V rows read,
   2 * sum(len_b) * Hkv * D * 2.
 
+``e2e``: the same metrics through the public API with the inputs in pinned
+host memory.  Prefill copies each step's q, k, v and positions in and the
+output out, pipelined over three streams; decode keeps the caches resident
+(model state) and copies each step's q, lengths and positions in and the
+output out, steps in sequence on one stream.
+
 ``--phase configs`` instead times every named workload (the five shapes the
 parity tests cover) through the public API, one JSON line per workload, with
 CUDA events around each call (direct launches); it is a report, not the
