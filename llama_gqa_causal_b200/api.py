@@ -133,6 +133,30 @@ def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
     return t.data_ptr()
 
 
+def _need(t: Optional[torch.Tensor], where: str, name: str, dtype: torch.dtype,
+          device: torch.device, shape=None, numel: Optional[int] = None) -> None:
+    """Reject a tensor whose dtype, device or size disagrees with the sizes the
+    entry point is given (the C ABI sees only pointers: a short buffer would be
+    read or written past its end)."""
+    if t is None:
+        return
+    if t.dtype != dtype:
+        raise ValueError(f"{where}: {name} must be {dtype}, got {t.dtype}")
+    if t.device != device:
+        raise ValueError(f"{where}: {name} is on {t.device}, expected {device}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{where}: {name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if numel is not None and t.numel() != numel:
+        raise ValueError(f"{where}: {name} must hold {numel} elements, got {t.numel()}")
+
+
+def _tables(cos, sin, where, device, rows, D) -> None:
+    if (cos is None) != (sin is None):
+        raise ValueError(f"{where}: pass both cos and sin, or neither")
+    _need(cos, where, "cos", torch.float32, device, numel=rows * D)
+    _need(sin, where, "sin", torch.float32, device, numel=rows * D)
+
+
 def _stream(stream=None) -> int:
     s = torch.cuda.current_stream() if stream is None else stream
     return s.cuda_stream
@@ -183,12 +207,18 @@ def qkv_rope(x: torch.Tensor, w_qkv: torch.Tensor, n_heads: int, n_kv_heads: int
     """llama_attn_qkv_rope.  x [T, hidden], w_qkv [(H+2Hkv)D, hidden] -> q [T,H,D], k, v [T,Hkv,D]."""
     lib = load()
     T, hidden = x.shape
+    w = "llama_attn_qkv_rope"
+    _need(w_qkv, w, "w_qkv", x.dtype, x.device, shape=((n_heads + 2 * n_kv_heads) * head_dim, hidden))
+    _tables(cos, sin, w, x.device, T, head_dim)
     if out is None:
         q = torch.empty(T, n_heads, head_dim, device=x.device, dtype=x.dtype)
         k = torch.empty(T, n_kv_heads, head_dim, device=x.device, dtype=x.dtype)
         v = torch.empty_like(k)
     else:
         q, k, v = out
+        _need(q, w, "q", x.dtype, x.device, numel=T * n_heads * head_dim)
+        _need(k, w, "k", x.dtype, x.device, numel=T * n_kv_heads * head_dim)
+        _need(v, w, "v", x.dtype, x.device, numel=T * n_kv_heads * head_dim)
     _check(lib.llama_attn_qkv_rope(_ptr(x), _ptr(w_qkv), _ptr(cos), _ptr(sin), T, hidden, n_heads,
                                    n_kv_heads, head_dim, _ptr(q), _ptr(k), _ptr(v),
                                    _dtype_code(x.dtype), _stream(stream)), "llama_attn_qkv_rope")
@@ -202,8 +232,10 @@ def out_proj(attn: torch.Tensor, w_o: torch.Tensor, *, out: Optional[torch.Tenso
     attn2 = attn.reshape(attn.shape[0], -1)
     T, d_in = attn2.shape
     d_out = w_o.shape[0]
+    _need(w_o, "llama_attn_out_proj", "w_o", attn.dtype, attn.device, shape=(d_out, d_in))
     if out is None:
         out = torch.empty(T, d_out, device=attn.device, dtype=attn.dtype)
+    _need(out, "llama_attn_out_proj", "out", attn.dtype, attn.device, numel=T * d_out)
     _check(lib.llama_attn_out_proj(_ptr(attn2), _ptr(w_o), T, d_in, d_out, _ptr(out),
                                    _dtype_code(attn.dtype), _stream(stream)), "llama_attn_out_proj")
     return out
@@ -227,6 +259,11 @@ def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
     lib = load()
     b, S, H, D = q.shape
     Hkv = k.shape[2]
+    _need(k, "llama_attn_prefill", "k", q.dtype, q.device, shape=(b, S, Hkv, D))
+    _need(v, "llama_attn_prefill", "v", q.dtype, q.device, shape=(b, S, Hkv, D))
+    _tables(cos, sin, "llama_attn_prefill", q.device, b * S, D)
+    _need(out, "llama_attn_prefill", "out", q.dtype, q.device, numel=b * S * H * D)
+    _need(mask, "llama_attn_prefill", "mask", torch.float32, q.device, numel=b * S * S)
     if scale is None:
         scale = 1.0 / math.sqrt(D)
     if out is None:
@@ -251,6 +288,10 @@ def prefill_window(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
     lib = load()
     b, S, H, D = q.shape
     Hkv = k.shape[2]
+    _need(k, "llama_attn_prefill_window", "k", q.dtype, q.device, shape=(b, S, Hkv, D))
+    _need(v, "llama_attn_prefill_window", "v", q.dtype, q.device, shape=(b, S, Hkv, D))
+    _tables(cos, sin, "llama_attn_prefill_window", q.device, b * S, D)
+    _need(out, "llama_attn_prefill_window", "out", q.dtype, q.device, numel=b * S * H * D)
     if scale is None:
         scale = 1.0 / math.sqrt(D)
     if out is None:
@@ -275,6 +316,11 @@ def prefill_varlen(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, seq_lens: 
     lib = load()
     b, S, H, D = q.shape
     Hkv = k.shape[2]
+    _need(k, "llama_attn_prefill_varlen", "k", q.dtype, q.device, shape=(b, S, Hkv, D))
+    _need(v, "llama_attn_prefill_varlen", "v", q.dtype, q.device, shape=(b, S, Hkv, D))
+    _tables(cos, sin, "llama_attn_prefill_varlen", q.device, b * S, D)
+    _need(out, "llama_attn_prefill_varlen", "out", q.dtype, q.device, numel=b * S * H * D)
+    _need(seq_lens, "llama_attn_prefill_varlen", "seq_lens", torch.int32, q.device, numel=b)
     if scale is None:
         scale = 1.0 / math.sqrt(D)
     if seq_lens.dtype != torch.int32:
@@ -303,6 +349,12 @@ def prefill_packed(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlens
     T, H, D = q.shape
     Hkv = k.shape[1]
     n = cu_seqlens.numel() - 1
+    w = "llama_attn_prefill_packed"
+    _need(k, w, "k", q.dtype, q.device, shape=(T, Hkv, D))
+    _need(v, w, "v", q.dtype, q.device, shape=(T, Hkv, D))
+    _tables(cos, sin, w, q.device, T, D)
+    _need(out, w, "out", q.dtype, q.device, numel=T * H * D)
+    _need(cu_seqlens, w, "cu_seqlens", torch.int32, q.device)
     if scale is None:
         scale = 1.0 / math.sqrt(D)
     if cu_seqlens.dtype != torch.int32:
@@ -330,6 +382,11 @@ def decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
     lib = load()
     b, H, D = q.shape
     Hkv, L = k_cache.shape[1], k_cache.shape[2]
+    _need(k_cache, "llama_attn_decode", "k_cache", q.dtype, q.device, shape=(b, Hkv, L, D))
+    _need(v_cache, "llama_attn_decode", "v_cache", q.dtype, q.device, shape=(b, Hkv, L, D))
+    _need(cache_lens, "llama_attn_decode", "cache_lens", torch.int32, q.device, numel=b)
+    _tables(cos, sin, "llama_attn_decode", q.device, b, D)
+    _need(out, "llama_attn_decode", "out", q.dtype, q.device, numel=b * H * D)
     if scale is None:
         scale = 1.0 / math.sqrt(D)
     if out is None:
@@ -358,6 +415,11 @@ def decode_append(q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor,
     lib = load()
     b, H, D = q.shape
     Hkv, L = k_cache.shape[1], k_cache.shape[2]
+    _need(k_cache, "llama_attn_decode_append", "k_cache", q.dtype, q.device, shape=(b, Hkv, L, D))
+    _need(v_cache, "llama_attn_decode_append", "v_cache", q.dtype, q.device, shape=(b, Hkv, L, D))
+    _need(cache_lens, "llama_attn_decode_append", "cache_lens", torch.int32, q.device, numel=b)
+    _tables(cos, sin, "llama_attn_decode_append", q.device, b, D)
+    _need(out, "llama_attn_decode_append", "out", q.dtype, q.device, numel=b * H * D)
     if scale is None:
         scale = 1.0 / math.sqrt(D)
     if out is None:
@@ -391,6 +453,11 @@ def decode_noalloc(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor
     lib = load()
     b, H, D = q.shape
     Hkv, L = k_cache.shape[1], k_cache.shape[2]
+    _need(k_cache, "llama_attn_decode_noalloc", "k_cache", q.dtype, q.device, shape=(b, Hkv, L, D))
+    _need(v_cache, "llama_attn_decode_noalloc", "v_cache", q.dtype, q.device, shape=(b, Hkv, L, D))
+    _need(cache_lens, "llama_attn_decode_noalloc", "cache_lens", torch.int32, q.device, numel=b)
+    _tables(cos, sin, "llama_attn_decode_noalloc", q.device, b, D)
+    _need(out, "llama_attn_decode_noalloc", "out", q.dtype, q.device, numel=b * H * D)
     if scale is None:
         scale = 1.0 / math.sqrt(D)
     if cache_lens.dtype != torch.int32:

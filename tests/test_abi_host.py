@@ -323,3 +323,45 @@ def test_loader_fails_loudly_without_the_library(tmp_path, monkeypatch):
         api.rope_table(torch.zeros(1, 4, dtype=torch.int64), 128)
     monkeypatch.undo()
     assert api.load() is not None
+
+
+def _bf(*shape):
+    return torch.zeros(*shape, dtype=torch.bfloat16)
+
+
+@pytest.mark.parametrize("call,match", [
+    (lambda: api.prefill(_bf(1, 8, 4, 64), _bf(1, 7, 2, 64), _bf(1, 8, 2, 64)), "k must have shape"),
+    (lambda: api.prefill(_bf(1, 8, 4, 64), _bf(1, 8, 2, 64), _bf(1, 8, 2, 64).float()),
+     "v must be torch.bfloat16"),
+    (lambda: api.prefill(_bf(1, 8, 4, 64), _bf(1, 8, 2, 64), _bf(1, 8, 2, 64),
+                         torch.zeros(1, 8, 64)), "both cos and sin"),
+    (lambda: api.prefill(_bf(1, 8, 4, 64), _bf(1, 8, 2, 64), _bf(1, 8, 2, 64),
+                         torch.zeros(1, 8, 32), torch.zeros(1, 8, 32)), "cos must hold 512"),
+    (lambda: api.prefill(_bf(1, 8, 4, 64), _bf(1, 8, 2, 64), _bf(1, 8, 2, 64),
+                         mask=torch.zeros(1, 1, 8, 7)), "mask must hold 64"),
+    (lambda: api.prefill(_bf(1, 8, 4, 64), _bf(1, 8, 2, 64), _bf(1, 8, 2, 64),
+                         out=_bf(1, 8, 128)), "out must hold 2048"),
+    (lambda: api.prefill_window(_bf(1, 8, 4, 64), _bf(1, 8, 2, 64), _bf(1, 8, 1, 64), window=4),
+     "v must have shape"),
+    (lambda: api.prefill_varlen(_bf(2, 8, 4, 64), _bf(2, 8, 2, 64), _bf(2, 8, 2, 64),
+                                torch.zeros(3, dtype=torch.int32)), "seq_lens must hold 2"),
+    (lambda: api.prefill_packed(_bf(10, 4, 64), _bf(9, 2, 64), _bf(10, 2, 64),
+                                torch.tensor([0, 10], dtype=torch.int32), 10), "k must have shape"),
+    (lambda: api.decode(_bf(2, 8, 64), _bf(2, 2, 16, 64), _bf(2, 2, 15, 64),
+                        torch.zeros(2, dtype=torch.int32)), "v_cache must have shape"),
+    (lambda: api.decode(_bf(2, 8, 64), _bf(2, 2, 16, 64), _bf(2, 2, 16, 64),
+                        torch.zeros(2, dtype=torch.int64)), "cache_lens must be torch.int32"),
+    (lambda: api.decode_append(_bf(2, 8, 64), _bf(2, 2, 64), _bf(2, 2, 64), _bf(2, 2, 16, 64),
+                               _bf(2, 2, 16, 64), torch.zeros(1, dtype=torch.int32)),
+     "cache_lens must hold 2"),
+    (lambda: api.decode_noalloc(_bf(2, 8, 64), _bf(2, 2, 16, 64), _bf(2, 2, 16, 64),
+                                torch.zeros(2, dtype=torch.int32), out=_bf(2, 256)),
+     "out must hold 1024"),
+    (lambda: api.qkv_rope(_bf(5, 32), _bf(3 * 64, 32), 2, 1, 64), "w_qkv must have shape"),
+    (lambda: api.out_proj(_bf(5, 32), _bf(16, 31)), "w_o must have shape"),
+])
+def test_python_binding_checks_tensor_sizes_before_any_launch(lib, call, match):
+    # the C ABI sees only pointers: the binding refuses tensors that disagree
+    # with the sizes it passes (checked before the device check, so on CPU here)
+    with pytest.raises(ValueError, match=match):
+        call()
