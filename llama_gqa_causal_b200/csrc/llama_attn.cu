@@ -282,8 +282,11 @@ int decode_bf16(const void* q, const void* kc, const void* vc, const int* lens, 
   const size_t smem = sizeof(la::DecSmem<D>) + 1024;
   const int append = (k_new != nullptr) ? 1 : 0;
   // Both kernels launch as programmatic dependents of what precedes them on
-  // the stream: their blocks are scheduled while the previous grid drains and
-  // wait on the device (griddepcontrol.wait) before touching global memory.
+  // the stream, so their blocks are scheduled while the previous grid drains.
+  // The split kernel waits on the device (griddepcontrol.wait) before it
+  // touches global memory; the combine reads only cache_lens before its own
+  // wait, which is final by then (it is scheduled only after every split CTA
+  // has passed its wait, so whatever wrote the lengths has finished).
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
