@@ -365,3 +365,30 @@ def test_python_binding_checks_tensor_sizes_before_any_launch(lib, call, match):
     # with the sizes it passes (checked before the device check, so on CPU here)
     with pytest.raises(ValueError, match=match):
         call()
+
+
+def test_header_is_plain_c_and_links(lib, tmp_path):
+    # the boundary is a C ABI: a strict C99 program includes the header, links
+    # against the library and calls its host-only entry points
+    import shutil
+    import subprocess
+    if shutil.which("gcc") is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "abi.c"
+    src.write_text(
+        "#include <stdio.h>\n#include \"llama_attn.h\"\n"
+        "int main(void) {\n"
+        "  printf(\"%d|%s|%zu\\n\", llama_attn_abi_version(),\n"
+        "         llama_attn_status_string(LLAMA_ERR_UNSUPPORTED),\n"
+        "         llama_attn_decode_workspace_bytes(32, 64, 4096, 128));\n"
+        "  return 0;\n}\n")
+    libdir = os.path.dirname(build.LIB)
+    exe = tmp_path / "abi"
+    subprocess.run(["gcc", "-std=c99", "-Wall", "-Wextra", "-Werror", "-pedantic",
+                    "-I", build.INCLUDE, str(src), "-L", libdir, "-lllama_attn",
+                    f"-Wl,-rpath,{libdir}", "-o", str(exe)], check=True)
+    out = subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.strip()
+    version, status, ws = out.split("|")
+    assert int(version) == lib.llama_attn_abi_version()
+    assert status == api.status_string(api.LLAMA_ERR_UNSUPPORTED)
+    assert int(ws) == api.decode_workspace_bytes(32, 64, 4096, 128)
