@@ -30,7 +30,8 @@
  *   llama_attn_decode           one query token per sequence against a KV cache
  *   llama_attn_decode_append    the same step with the token's own K/V appended
  *   llama_attn_decode_noalloc   decode on a static scratch (no caller workspace)
- *   plus workspace sizes, the device status word, status strings, ABI version.
+ *   plus workspace sizes, the device status word, failure-detection
+ *   self-tests, status strings, ABI version.
  *
  * Conventions shared by every entry point:
  *   - All tensor pointers are DEVICE pointers, contiguous, row-major, owned by
@@ -307,9 +308,10 @@ int llama_attn_decode_append(const void* q, const void* k_new, const void* v_new
  * more than that (see llama_attn_decode_workspace_bytes) is rejected with
  * LLAMA_ERR_INVALID_ARG before anything is enqueued; use llama_attn_decode
  * with a caller workspace instead.  fp32 requests need no scratch.
- * The first call on a device looks up the array's device address (one
- * cudaGetSymbolAddress, no allocation); make that first call before any
- * stream capture on that device.
+ * Every call looks up the array's device address on the current device (one
+ * cudaGetSymbolAddress, which allocates nothing).  The first call on a device
+ * may load the library's device code there: make it before any stream
+ * capture on that device.
  * Every call on a device shares the one array and leaves its last contents
  * behind (each call writes every scratch entry it later reads, so nothing has
  * to start at zero).  Calls whose kernels overlap on the GPU -- concurrent
@@ -325,10 +327,32 @@ int llama_attn_decode_noalloc(const void* q, const void* k_cache, const void* v_
  * LLAMA_ERR_CUDA if the synchronisation itself failed. */
 int llama_attn_device_status(void* cuda_stream);
 
+/*
+ * Self-tests of failure detection.  The pages have no counterpart; these two
+ * calls let a test (or a deployment's health check) see both failure paths
+ * of the library work without faulting the GPU.
+ *
+ * llama_attn_selftest_wait_timeout: launches one warp that waits on a shared-
+ * memory barrier nothing ever arrives on, with the given limit in
+ * microseconds (1 .. 1000000) instead of the pipelines' 2 s.  The wait runs
+ * out, records LLAMA_ERR_DEVICE_TIMEOUT in the device status word and the
+ * kernel returns, with no copy or MMA in flight.  Returns LLAMA_OK once the
+ * launch is enqueued (INVALID_ARG for a limit outside the range); a following
+ * llama_attn_device_status() reports LLAMA_ERR_DEVICE_TIMEOUT, the next one
+ * LLAMA_OK.
+ *
+ * llama_attn_selftest_launch_error: asks for a kernel launch with an invalid
+ * block size, which the CUDA runtime refuses on the host; returns
+ * LLAMA_ERR_CUDA, as any library call whose launch fails does.  Nothing
+ * reaches the GPU and the context stays usable.
+ */
+int llama_attn_selftest_wait_timeout(unsigned int limit_us, void* cuda_stream);
+int llama_attn_selftest_launch_error(void* cuda_stream);
+
 /* Static, NUL-terminated description of a status code. */
 const char* llama_attn_status_string(int status);
 
-/* ABI version (major * 100 + minor): 110 = 1.1, the entry points above. */
+/* ABI version (major * 100 + minor): 120 = 1.2, the entry points above. */
 int llama_attn_abi_version(void);
 
 #ifdef __cplusplus

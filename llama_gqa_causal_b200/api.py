@@ -45,6 +45,8 @@ EXPORTED = (
     "llama_attn_decode_append",
     "llama_attn_decode_noalloc",
     "llama_attn_device_status",
+    "llama_attn_selftest_wait_timeout",
+    "llama_attn_selftest_launch_error",
     "llama_attn_status_string",
     "llama_attn_abi_version",
 )
@@ -106,6 +108,10 @@ def load() -> ctypes.CDLL:
     lib.llama_attn_decode_noalloc.restype = I
     lib.llama_attn_device_status.argtypes = [P]
     lib.llama_attn_device_status.restype = I
+    lib.llama_attn_selftest_wait_timeout.argtypes = [ctypes.c_uint, P]
+    lib.llama_attn_selftest_wait_timeout.restype = I
+    lib.llama_attn_selftest_launch_error.argtypes = [P]
+    lib.llama_attn_selftest_launch_error.restype = I
     lib.llama_attn_status_string.argtypes = [I]
     lib.llama_attn_status_string.restype = ctypes.c_char_p
     lib.llama_attn_abi_version.argtypes = []
@@ -472,3 +478,13 @@ def decode_noalloc(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor
 def device_status(stream=None) -> int:
     """llama_attn_device_status: sync the stream, read and clear the device status word."""
     return int(load().llama_attn_device_status(_stream(stream)))
+
+
+def selftest_wait_timeout(limit_us: int, stream=None) -> int:
+    """llama_attn_selftest_wait_timeout: a bounded device wait that runs out (status code)."""
+    return int(load().llama_attn_selftest_wait_timeout(int(limit_us), _stream(stream)))
+
+
+def selftest_launch_error(stream=None) -> int:
+    """llama_attn_selftest_launch_error: a launch the runtime refuses (status code)."""
+    return int(load().llama_attn_selftest_launch_error(_stream(stream)))

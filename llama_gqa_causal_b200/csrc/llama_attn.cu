@@ -20,7 +20,7 @@
 
 namespace {
 
-constexpr int kAbiVersion = 110;
+constexpr int kAbiVersion = 120;
 
 // ---------------------------------------------------------------- host helpers
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -331,6 +331,22 @@ int decode_bf16(const void* q, const void* kc, const void* vc, const int* lens, 
   return launch_status();
 }
 
+// ---------------------------------------------------------------- failure-detection self-tests
+// A warp waits on an mbarrier that nothing ever arrives on, with a short
+// limit: the wait runs out, records the timeout in the device status word
+// and the kernel returns.  No copy or MMA is in flight, so the context stays
+// usable; this is the path every pipeline wait of the library takes on expiry.
+__global__ void selftest_wait_timeout_kernel(unsigned long long limit_ns) {
+  __shared__ uint64_t never_armed;
+  if (threadIdx.x == 0) {
+    la::mbar_init(&never_armed, 1);
+    la::fence_mbar_init();
+  }
+  __syncthreads();
+  la::mbar_wait(&never_armed, 0, limit_ns);
+}
+__global__ void selftest_noop_kernel() {}
+
 }  // namespace
 
 // ---------------------------------------------------------------- decode without caller scratch
@@ -345,21 +361,14 @@ static __device__ __align__(256) unsigned char g_decode_noalloc_scratch[kNoAlloc
 
 namespace {
 // Device address of the scratch array on the current device.  Host code may
-// not use the array's name as a pointer (on the host it is only a stand-in
-// for the symbol), so the address is looked up once per device, with that
-// device current, and cached.
+// not use the array's name as a pointer (on the host it only stands for the
+// symbol), so the address is looked up with that device current, on every
+// call: an address kept from an earlier call would be stale once a device
+// reset has reloaded the library's device code.  The lookup allocates nothing.
 void* noalloc_scratch_for_current_device() {
-  static std::mutex mu;
-  static void* addr[64] = {};
-  int dev = -1;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-  std::lock_guard<std::mutex> lock(mu);
-  if (addr[dev] == nullptr) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_decode_noalloc_scratch) != cudaSuccess) return nullptr;
-    addr[dev] = p;
-  }
-  return addr[dev];
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_decode_noalloc_scratch) != cudaSuccess) return nullptr;
+  return p;
 }
 }  // namespace
 
@@ -649,6 +658,20 @@ int llama_attn_decode_noalloc(const void* q, const void* k_cache, const void* v_
   return llama_attn_decode(q, k_cache, v_cache, cache_lens, cos, sin, bsz, n_heads, n_kv_heads,
                            max_cache_len, head_dim, scale, out, scratch,
                            scratch ? kNoAllocScratchBytes : 0, dtype, cuda_stream);
+}
+
+int llama_attn_selftest_wait_timeout(unsigned int limit_us, void* cuda_stream) {
+  if (limit_us < 1 || limit_us > 1000000u) return LLAMA_ERR_INVALID_ARG;
+  selftest_wait_timeout_kernel<<<1, 32, 0, as_stream(cuda_stream)>>>(
+      static_cast<unsigned long long>(limit_us) * 1000ull);
+  return launch_status();
+}
+
+int llama_attn_selftest_launch_error(void* cuda_stream) {
+  // 2048 threads per block exceeds the 1024 every CUDA device allows: the
+  // runtime refuses the launch on the host, before anything reaches the GPU
+  selftest_noop_kernel<<<1, 2048, 0, as_stream(cuda_stream)>>>();
+  return launch_status();
 }
 
 int llama_attn_device_status(void* cuda_stream) {

@@ -42,7 +42,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_abi_version_and_status_strings(lib):
-    assert lib.llama_attn_abi_version() == 110
+    assert lib.llama_attn_abi_version() == 120
     assert api.status_string(0) == "ok"
     assert "invalid" in api.status_string(1)
     assert "unsupported" in api.status_string(2)
@@ -392,3 +392,8 @@ def test_header_is_plain_c_and_links(lib, tmp_path):
     assert int(version) == lib.llama_attn_abi_version()
     assert status == api.status_string(api.LLAMA_ERR_UNSUPPORTED)
     assert int(ws) == api.decode_workspace_bytes(32, 64, 4096, 128)
+
+
+@pytest.mark.parametrize("limit_us", [0, 1000001, 1 << 31])
+def test_selftest_wait_timeout_rejects_limits_outside_its_range(lib, limit_us):
+    assert lib.llama_attn_selftest_wait_timeout(limit_us, None) == api.LLAMA_ERR_INVALID_ARG
