@@ -376,6 +376,23 @@ def _prefill_phase(args, ws, local, dev, stream, line):
     return args.steps * 3
 
 
+def _pack_step_inputs(tensors, dev):
+    """One device byte buffer holding `tensors` back to back (each at a 16-byte
+    aligned offset) and typed views of it, shaped like the inputs."""
+    offs, total = [], 0
+    for t in tensors:
+        offs.append(total)
+        total += (t.numel() * t.element_size() + 15) // 16 * 16
+    stage = torch.empty(total, dtype=torch.uint8, device=dev)
+    views = []
+    for t, o in zip(tensors, offs):
+        n = t.numel() * t.element_size()
+        v = stage[o:o + n].view(t.dtype).view(t.shape)
+        v.copy_(t.to(dev))
+        views.append(v)
+    return stage, views
+
+
 def _decode_phase(args, ws, local, dev, stream, line):
     from llama_gqa_causal_b200 import api
     peak_burst, peak_sus, hbm, peak_src = _peaks()
@@ -383,7 +400,12 @@ def _decode_phase(args, ws, local, dev, stream, line):
     insts = []
     for rep in range(2):  # two caches, alternated, so no step reads L2-resident data
         y = W.decode_inputs(dcfg)
-        insts.append({n: y[n].to(dev) for n in ("q", "k_cache", "v_cache", "lens", "qpos")})
+        d = {n: y[n].to(dev) for n in ("k_cache", "v_cache")}
+        # a step's own inputs (q, lengths, positions) sit in one staging buffer,
+        # so the end-to-end run copies them in with a single transfer
+        d["stage"], views = _pack_step_inputs([y["q"], y["lens"], y["qpos"]], dev)
+        d["q"], d["lens"], d["qpos"] = views
+        insts.append(d)
     lens_cpu = y["lens"].to(torch.int64)
     dbytes = int(2 * lens_cpu.sum().item() * dcfg.n_kv_heads * dcfg.head_dim * 2)
     dout = torch.empty(dcfg.bsz, dcfg.n_heads * dcfg.head_dim, device=dev, dtype=dcfg.dtype)
@@ -436,13 +458,11 @@ def _decode_phase(args, ws, local, dev, stream, line):
     # after another on one stream.
     dec_e2e = None
     if not args.no_e2e:
-        hosts = [{n: insts[r][n].cpu().pin_memory() for n in ("q", "lens", "qpos")} for r in range(2)]
+        hosts = [insts[r]["stage"].cpu().pin_memory() for r in range(2)]
         hout = torch.empty(dout.shape, dtype=dout.dtype).pin_memory()
 
         def e2e_step(i):
-            d, h = insts[i % 2], hosts[i % 2]
-            for n in ("q", "lens", "qpos"):
-                d[n].copy_(h[n], non_blocking=True)
+            insts[i % 2]["stage"].copy_(hosts[i % 2], non_blocking=True)
             decode_step(i)
             hout.copy_(dout, non_blocking=True)
 
@@ -464,10 +484,11 @@ def _decode_phase(args, ws, local, dev, stream, line):
             "value": round(replicas.job_throughput(dbytes, dsteps, ms_e2e, ws) / 1e9, 1),
             "unit": "GB/s",
             "ms_per_step": round(ms_e2e / dsteps, 4),
-            "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in hosts[0].values()),
+            "h2d_bytes_per_step": hosts[0].numel() * hosts[0].element_size(),
             "d2h_bytes_per_step": hout.numel() * hout.element_size(),
             "steps": dsteps,
-            "launch": "one stream, steps in sequence, direct launches; caches resident",
+            "launch": "one stream, steps in sequence, direct launches; caches resident; the step's "
+                      "q, lengths and positions copied in as one pinned buffer",
         }
         del hosts, hout
 

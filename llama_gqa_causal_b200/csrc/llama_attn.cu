@@ -46,10 +46,63 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
+// A tensor map is a pure function of its base address, dimensions, strides
+// and box, so encoded maps are memoised: a decode loop that calls with the
+// same caches every step encodes its two maps once.  Small and
+// move-to-front; shared by all threads under a mutex.
+struct MapKey {
+  uintptr_t base;
+  int rank;
+  cuuint64_t dims[5];
+  cuuint64_t strides[4];
+  cuuint32_t box[5];
+  bool operator==(const MapKey& o) const {
+    if (base != o.base || rank != o.rank) return false;
+    for (int i = 0; i < rank; ++i)
+      if (dims[i] != o.dims[i] || box[i] != o.box[i]) return false;
+    for (int i = 0; i + 1 < rank; ++i)
+      if (strides[i] != o.strides[i]) return false;
+    return true;
+  }
+};
+struct MapCache {
+  static constexpr int kEntries = 32;
+  std::mutex mu;
+  int n = 0;
+  MapKey key[kEntries];
+  CUtensorMap map[kEntries];
+};
+MapCache& map_cache() {
+  static MapCache c;
+  return c;
+}
+
 // bf16 tensor map with the 128-byte swizzle; dims/strides innermost first
 // (strides in bytes, for dims 1..rank-1), box innermost first.
 bool make_map(CUtensorMap* m, const void* base, int rank, const cuuint64_t* dims,
               const cuuint64_t* strides, const cuuint32_t* box) {
+  MapKey k{};
+  k.base = reinterpret_cast<uintptr_t>(base);
+  k.rank = rank;
+  for (int i = 0; i < rank; ++i) {
+    k.dims[i] = dims[i];
+    k.box[i] = box[i];
+  }
+  for (int i = 0; i + 1 < rank; ++i) k.strides[i] = strides[i];
+  MapCache& c = map_cache();
+  {
+    std::lock_guard<std::mutex> lock(c.mu);
+    for (int i = 0; i < c.n; ++i) {
+      if (c.key[i] == k) {
+        *m = c.map[i];
+        for (int j = i; j > 0; --j) {  // move to the front
+          std::swap(c.key[j], c.key[j - 1]);
+          std::swap(c.map[j], c.map[j - 1]);
+        }
+        return true;
+      }
+    }
+  }
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   cuuint32_t estr[5] = {1, 1, 1, 1, 1};
@@ -57,7 +110,16 @@ bool make_map(CUtensorMap* m, const void* base, int rank, const cuuint64_t* dims
                   const_cast<void*>(base), dims, strides, box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
+  if (r != CUDA_SUCCESS) return false;
+  std::lock_guard<std::mutex> lock(c.mu);
+  const int last = c.n < MapCache::kEntries ? c.n++ : MapCache::kEntries - 1;  // evict the oldest
+  for (int j = last; j > 0; --j) {
+    c.key[j] = c.key[j - 1];
+    c.map[j] = c.map[j - 1];
+  }
+  c.key[0] = k;
+  c.map[0] = *m;
+  return true;
 }
 
 // Dynamic shared memory opt-in, once per (kernel, device).  Templated on the
