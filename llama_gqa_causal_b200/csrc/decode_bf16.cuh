@@ -50,6 +50,11 @@ constexpr int MAX_BATCH = 4096;  // per-batch chunk prefix lives in shared memor
 constexpr int MAX_CTAS = 256;    // persistent grid size cap (one CTA per SM)
 // floats per partial row: D outputs, then max and sum; padded to 16 bytes
 __host__ __device__ constexpr int part_stride(int d) { return d + 4; }
+// Bytes of the workspace's last region: the chunk prefix over the batch
+// ([bsz + 1] int32, written by the split kernel for the combine kernel).
+__host__ __device__ inline size_t ws_prefix_bytes(int bsz) {
+  return ((static_cast<size_t>(bsz) + 1) * 4 + 255) / 256 * 256;
+}
 }  // namespace dec
 
 struct DecodeParams {
@@ -63,6 +68,7 @@ struct DecodeParams {
   __nv_bfloat16* v_cache;
   float* ws_home;          // [b, H, D + 4]: partial of the segment at a sequence's start
   float* ws_cta;           // [MAX_CTAS, 8, D + 4]: partial of a CTA's mid-sequence segment
+  int* ws_prefix;          // [b + 1]: chunk prefix, written by CTA 0 for the combine kernel
   int bsz, H, Hkv, L, group, hchunks;
   float scale_log2;        // scale * log2(e)
 };
@@ -206,6 +212,9 @@ __global__ void __launch_bounds__(dec::THREADS, 1) decode_bf16_kernel(
       acc += (attend_len(p.lens[b], p.L, APPEND) + CH - 1) / CH;
     }
     __syncthreads();
+    // the combine kernel reads the prefix once this grid has finished
+    if (blockIdx.x == 0)
+      for (int b = threadIdx.x; b <= p.bsz; b += THREADS) p.ws_prefix[b] = s.chunk_prefix[b];
   }
   // the combine kernel may be scheduled now; it waits for this grid to finish
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -514,52 +523,31 @@ __global__ void __launch_bounds__(dec::THREADS, 1) decode_bf16_kernel(
 // The sequence's segments start at its first chunk (home slot) and at every
 // chunk where some CTA's share begins inside it (that CTA's own slot).
 //   m* = max_s m_s,  l = sum_s l_s 2^(m_s - m*),  o = sum_s o_s 2^(m_s - m*) / l.
-// Everything that depends only on cache_lens (the chunk prefix of the batch
-// entry, the segment starts) is computed before the wait for the split kernel,
-// and the partials of up to kEager segments are then loaded at once.
+// The chunk prefix of the batch comes from the split kernel through the
+// workspace and, like everything else that grid wrote, is read only after the
+// wait for it; the partials of up to kEager segments are then loaded at once.
 namespace dec {
 constexpr int COMBINE_THREADS = 256;  // 8 warps = the heads of one sequence
 }
 template <int D>
 __global__ void __launch_bounds__(dec::COMBINE_THREADS) decode_combine_kernel(
-    const float* __restrict__ ws_home, const float* __restrict__ ws_cta,
-    const int* __restrict__ lens, __nv_bfloat16* __restrict__ out, int bsz, int H, int Hkv, int L,
-    int group, int hchunks, int n_ctas, int append) {
+    const float* ws_home, const float* ws_cta, const int* ws_prefix,
+    __nv_bfloat16* __restrict__ out, int bsz, int H, int Hkv, int group, int hchunks,
+    int n_ctas) {
   constexpr int kEager = 4;
   constexpr int VEC = D / 32;  // dimensions per lane
-  constexpr int NW = dec::COMBINE_THREADS / 32;
   const int seq = blockIdx.x, b = blockIdx.y;
   const int kvh = seq / hchunks, hc = seq - kvh * hchunks;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   // a programmatic dependent launched after this kernel (the next decode) may
   // be scheduled now; it waits for this grid to finish before touching memory
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-  // chunks of batch entries < b and of all entries: block-wide sums over lens
-  __shared__ long long red[2][NW];
-  long long before = 0, all = 0;
-  for (int e = threadIdx.x; e < bsz; e += dec::COMBINE_THREADS) {
-    const int c = (attend_len(lens[e], L, append) + dec::CH - 1) / dec::CH;
-    all += c;
-    if (e < b) before += c;
-  }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    before += __shfl_xor_sync(0xffffffffu, before, o);
-    all += __shfl_xor_sync(0xffffffffu, all, o);
-  }
-  if (lane == 0) {
-    red[0][warp] = before;
-    red[1][warp] = all;
-  }
-  __syncthreads();
-  long long prefix_b = 0, total = 0;
-#pragma unroll
-  for (int w = 0; w < NW; ++w) {
-    prefix_b += red[0][w];
-    total += red[1][w];
-  }
+  // the split kernel's writes (prefix and partials) are visible after this
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  const long long prefix_b = ws_prefix[b];
+  const long long total = ws_prefix[bsz];
   const int per_b = Hkv * hchunks;
-  const int nch = (attend_len(lens[b], L, append) + dec::CH - 1) / dec::CH;
+  const int nch = static_cast<int>(ws_prefix[b + 1] - prefix_b);
   const long long n_chunks = total * per_b;
   const long long G = n_ctas;
   const long long P = prefix_b * per_b + static_cast<long long>(seq) * nch;
@@ -584,11 +572,8 @@ __global__ void __launch_bounds__(dec::COMBINE_THREADS) decode_combine_kernel(
   for (int k = 0; k < kEager; ++k) own[k] = next_owner();
 
   const int hq = hc * 8 + warp;  // query head within the group
-  const bool active = hq < group;
+  if (hq >= group) return;
   const int head = kvh * group + hq;
-  // the split kernel's writes are visible after this (programmatic dependent launch)
-  asm volatile("griddepcontrol.wait;" ::: "memory");
-  if (!active) return;
   float mstar = -INFINITY, lsum = 0.f, acc[VEC];
 #pragma unroll
   for (int v = 0; v < VEC; ++v) acc[v] = 0.f;

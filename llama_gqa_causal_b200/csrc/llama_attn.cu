@@ -334,6 +334,8 @@ int decode_bf16(const void* q, const void* kc, const void* vc, const int* lens, 
   p.v_cache = static_cast<__nv_bfloat16*>(const_cast<void*>(vc));
   p.ws_home = static_cast<float*>(workspace);
   p.ws_cta = p.ws_home + static_cast<size_t>(bsz) * H * la::dec::part_stride(D);
+  p.ws_prefix = reinterpret_cast<int*>(p.ws_cta + static_cast<size_t>(la::dec::MAX_CTAS) * 8 *
+                                                      la::dec::part_stride(D));
   p.bsz = bsz;
   p.H = H;
   p.Hkv = Hkv;
@@ -345,10 +347,8 @@ int decode_bf16(const void* q, const void* kc, const void* vc, const int* lens, 
   const int append = (k_new != nullptr) ? 1 : 0;
   // Both kernels launch as programmatic dependents of what precedes them on
   // the stream, so their blocks are scheduled while the previous grid drains.
-  // The split kernel waits on the device (griddepcontrol.wait) before it
-  // touches global memory; the combine reads only cache_lens before its own
-  // wait, which is final by then (it is scheduled only after every split CTA
-  // has passed its wait, so whatever wrote the lengths has finished).
+  // Each waits on the device (griddepcontrol.wait) before it reads or writes
+  // global memory.
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
@@ -381,11 +381,11 @@ int decode_bf16(const void* q, const void* kc, const void* vc, const int* lens, 
   cfg.numAttrs = 1;
   const float* home = p.ws_home;
   const float* ctas = p.ws_cta;
+  const int* prefix = p.ws_prefix;
   __nv_bfloat16* o = static_cast<__nv_bfloat16*>(out);
   int group = p.group, hchunks = p.hchunks;
   const cudaError_t e = cudaLaunchKernelEx(&cfg, la::decode_combine_kernel<D>, home, ctas,
-                                           lens, o, bsz, H, Hkv, L, group, hchunks, n_ctas,
-                                           append);
+                                           prefix, o, bsz, H, Hkv, group, hchunks, n_ctas);
   if (e != cudaSuccess) {
     fprintf(stderr, "llama_attn: combine launch failed: %s\n", cudaGetErrorString(e));
     return LLAMA_ERR_CUDA;
@@ -629,9 +629,10 @@ int llama_attn_prefill_packed(const void* q, const void* k, const void* v, const
 
 size_t llama_attn_decode_workspace_bytes(int bsz, int n_heads, int max_cache_len, int head_dim) {
   if (bsz < 1 || n_heads < 1 || max_cache_len < 1 || head_dim < 1) return 0;
-  // one partial per (batch, head) plus one per (CTA, head of an 8-head chunk)
+  // one partial per (batch, head) plus one per (CTA, head of an 8-head
+  // chunk), then the chunk prefix over the batch
   const size_t rows = static_cast<size_t>(bsz) * n_heads + static_cast<size_t>(la::dec::MAX_CTAS) * 8;
-  return rows * la::dec::part_stride(head_dim) * sizeof(float);
+  return rows * la::dec::part_stride(head_dim) * sizeof(float) + la::dec::ws_prefix_bytes(bsz);
 }
 
 int llama_attn_decode(const void* q, const void* k_cache, const void* v_cache,

@@ -57,10 +57,14 @@ def test_workspace_sizes(lib):
     assert lib.llama_attn_prefill_workspace_bytes(1, 64, 8, 8192, 128, 1, 0) == 0
     assert lib.llama_attn_prefill_workspace_bytes(1, 4, 2, 64, 64, 0, 1) == 0
     # decode: one partial row of D + 4 floats per (b, head) and per (CTA, head of
-    # an 8-head chunk) for up to 256 CTAs; independent of the cache length
-    assert lib.llama_attn_decode_workspace_bytes(32, 64, 4096, 128) == (32 * 64 + 256 * 8) * 132 * 4
-    assert lib.llama_attn_decode_workspace_bytes(2, 4, 513, 64) == (2 * 4 + 256 * 8) * 68 * 4
-    assert lib.llama_attn_decode_workspace_bytes(2, 4, 1 << 20, 64) == (2 * 4 + 256 * 8) * 68 * 4
+    # an 8-head chunk) for up to 256 CTAs, then the chunk prefix over the batch
+    # ([b + 1] int32 in 256-byte units); independent of the cache length
+    def dec(b, H, D):
+        return (b * H + 256 * 8) * (D + 4) * 4 + ((b + 1) * 4 + 255) // 256 * 256
+    assert lib.llama_attn_decode_workspace_bytes(32, 64, 4096, 128) == dec(32, 64, 128)
+    assert lib.llama_attn_decode_workspace_bytes(2, 4, 513, 64) == dec(2, 4, 64)
+    assert lib.llama_attn_decode_workspace_bytes(2, 4, 1 << 20, 64) == dec(2, 4, 64)
+    assert lib.llama_attn_decode_workspace_bytes(4096, 8, 64, 64) == dec(4096, 8, 64)
     assert lib.llama_attn_decode_workspace_bytes(0, 4, 513, 64) == 0
 
 

@@ -69,7 +69,7 @@ def test_noalloc_decode_matches_workspace_decode_on_two_calls():
 def test_noalloc_rejects_requests_beyond_its_static_scratch():
     lib = api.load()
     fake = 0x10000  # never dereferenced: the request is refused on the host
-    # (1024 x 64 heads + 2048) partial rows x 132 floats = 35.7 MB of scratch > 16 MiB
+    # (1024 x 64 heads + 2048) partial rows x 132 floats + the prefix = 35.7 MB > 16 MiB
     st = lib.llama_attn_decode_noalloc(fake, fake, fake, fake, None, None, 1024, 64, 8, 4096, 128,
                                        0.088, fake, api.LLAMA_DT_BF16, None)
     assert st == api.LLAMA_ERR_INVALID_ARG
