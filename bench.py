@@ -101,9 +101,12 @@ def _max_over_ranks(x: float, ws: int) -> float:
 # ----------------------------------------------------------------------------- clocks
 
 class ClockSampler:
-    """nvidia-smi sampling of SM clock and throttle reasons during a timed region."""
+    """nvidia-smi sampling (every 10 ms) of SM clock, power and throttle
+    reasons; `summary()` keeps only the samples taken inside the windows marked
+    with `mark()` (wall-clock spans in which the GPU runs the timed work), so
+    idle moments between phases do not dilute the figure."""
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
@@ -111,6 +114,7 @@ class ClockSampler:
         self.gpu = gpu_index
         self.proc = None
         self.path = None
+        self.windows = []
 
     def __enter__(self):
         fd, self.path = tempfile.mkstemp(suffix=".csv")
@@ -118,7 +122,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.FIELDS,
-                 "--format=csv,noheader,nounits", "-lms", "100"],
+                 "--format=csv,noheader,nounits", "-lms", "10"],
                 stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
             time.sleep(0.3)
         except Exception:
@@ -127,35 +131,46 @@ class ClockSampler:
 
     def __exit__(self, *exc):
         if self.proc is not None:
+            time.sleep(0.05)
             self.proc.terminate()
             try:
                 self.proc.wait(timeout=5)
             except Exception:
                 self.proc.kill()
 
+    def mark(self, t0: float, t1: float):
+        self.windows.append((t0, t1))
+
     def summary(self):
-        out = {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        import datetime
+        out = {"sm_mhz": None, "sm_max_mhz": None, "power_w": None, "reasons": [], "samples": 0,
+               "window_s": round(sum(b - a for a, b in self.windows), 4)}
         if not self.path or not os.path.exists(self.path):
             return out
         rows = []
         for line in open(self.path):
             f = [x.strip() for x in line.split(",")]
-            if len(f) < 9:
+            if len(f) < 10:
                 continue
             try:
-                rows.append((float(f[1]), float(f[2]), f[5], f[6], f[7], f[8]))
+                ts = datetime.datetime.strptime(f[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                rows.append((ts, float(f[2]), float(f[3]), float(f[4]), f[6], f[7], f[8], f[9]))
             except ValueError:
                 continue
         os.unlink(self.path)
+        if self.windows:
+            inside = [r for r in rows if any(a <= r[0] <= b for a, b in self.windows)]
+            rows = inside if inside else rows
         if not rows:
             return out
         out["samples"] = len(rows)
-        out["sm_mhz"] = statistics.median(r[0] for r in rows)
-        out["sm_max_mhz"] = max(r[1] for r in rows)
+        out["sm_mhz"] = statistics.median(r[1] for r in rows)
+        out["sm_max_mhz"] = max(r[2] for r in rows)
+        out["power_w"] = round(statistics.median(r[3] for r in rows), 1)
         names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
         reasons = set()
         for r in rows:
-            for n, v in zip(names, r[2:]):
+            for n, v in zip(names, r[4:]):
                 if v.lower() == "active":
                     reasons.add(n)
         out["reasons"] = sorted(reasons)
@@ -251,16 +266,20 @@ def _prefill_phase(args, ws, local, dev, stream, line):
             graph.replay() if graph is not None else prefill_step()
         _barrier(ws)
         torch.cuda.synchronize()
+        w0 = time.time()
         t0.record(stream)
         for i in range(args.steps):
             graph.replay() if graph is not None else prefill_step()
         t1.record(stream)
         torch.cuda.synchronize()
+        clk.mark(w0, time.time())
         _barrier(ws)
         # the prefill call alone, events around each call (roofline figure)
+        w0 = time.time()
         for i in range(args.steps):
             prefill_step(evs[i])
         torch.cuda.synchronize()
+        clk.mark(w0, time.time())
     clocks = clk.summary()
     ms_total = _max_over_ranks(t0.elapsed_time(t1), ws)
     ms_call = _max_over_ranks(statistics.mean(a.elapsed_time(b) for a, b in evs), ws)

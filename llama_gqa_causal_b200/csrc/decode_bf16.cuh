@@ -173,6 +173,13 @@ __global__ void __launch_bounds__(dec::THREADS, 1) decode_bf16_kernel(
     tma_prefetch_desc(&tm_k);
     tma_prefetch_desc(&tm_v);
   }
+  if (threadIdx.x == 0) {  // shared memory only: set up before the grid-dependency wait
+    for (int i = 0; i < NSTAGE; ++i) {
+      mbar_init(&s.full[i], 1);
+      mbar_init(&s.empty[i], NCW);
+    }
+    fence_mbar_init();
+  }
   // Launched as a programmatic dependent of whatever precedes it on the stream:
   // the CTAs may be resident before that grid has finished, so nothing in
   // global memory is read or written before this wait (the previous decode's
@@ -196,13 +203,6 @@ __global__ void __launch_bounds__(dec::THREADS, 1) decode_bf16_kernel(
       if (lane >= o) incl += y;
     }
     if (lane == 31) warp_total[warp] = incl;
-    if (threadIdx.x == 0) {
-      for (int i = 0; i < NSTAGE; ++i) {
-        mbar_init(&s.full[i], 1);
-        mbar_init(&s.empty[i], NCW);
-      }
-      fence_mbar_init();
-    }
     __syncthreads();
     int acc = incl - sum;  // exclusive prefix of this thread's run
     for (int w = 0; w < warp; ++w) acc += warp_total[w];

@@ -462,8 +462,14 @@ int llama_rope_table(const long long* pos, int bsz, int seq, int head_dim, doubl
   const int blocks =
       static_cast<int>(std::min<long long>((n + rows_per_block - 1) / rows_per_block, 148LL * 32));
   if (threads > 1024) return LLAMA_ERR_UNSUPPORTED;
+  // the inverse frequencies theta^(-2i/D), i < D/2, formed once here in
+  // double rather than by every thread of the kernel
+  la::RopeFreqs freqs{};
+  if (half <= la::kRopeHostFreqs)
+    for (int i = 0; i < half; ++i)
+      freqs.inv[i] = std::exp(-(2.0 * i / head_dim) * std::log(theta));
   la::rope_table_kernel<<<blocks, threads, 0, as_stream(cuda_stream)>>>(
-      pos, n, head_dim, theta, pos_scale_factor, cos, sin);
+      pos, n, head_dim, theta, pos_scale_factor, cos, sin, freqs);
   return launch_status();
 }
 

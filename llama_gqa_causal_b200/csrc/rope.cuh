@@ -16,9 +16,17 @@
 
 namespace la {
 
+// Inverse frequencies theta^(-2i/D) formed on the host (in double) for
+// head_dim <= 2 * kRopeHostFreqs, passed by value; 0 entries mean "form them
+// on the device".
+constexpr int kRopeHostFreqs = 64;
+struct RopeFreqs {
+  double inv[kRopeHostFreqs];
+};
+
 __global__ void rope_table_kernel(const long long* __restrict__ pos, long long n_rows, int D,
                                   double theta, double factor, float* __restrict__ cos_out,
-                                  float* __restrict__ sin_out) {
+                                  float* __restrict__ sin_out, const __grid_constant__ RopeFreqs freqs) {
   // blockDim.x is a multiple of D/2: each thread keeps one frequency index i
   // (so its inverse frequency is formed once) and walks the rows
   // a programmatic dependent launched after this kernel (a decode reading the
@@ -27,7 +35,8 @@ __global__ void rope_table_kernel(const long long* __restrict__ pos, long long n
   const int half = D / 2;
   const int i = static_cast<int>(threadIdx.x % half);
   const int rows_per_block = static_cast<int>(blockDim.x / half);
-  const double inv_freq = exp(-(2.0 * i / D) * log(theta));
+  const double inv_freq =
+      half <= kRopeHostFreqs ? freqs.inv[i] : exp(-(2.0 * i / D) * log(theta));
   for (long long r = blockIdx.x * (long long)rows_per_block + threadIdx.x / half; r < n_rows;
        r += (long long)gridDim.x * rows_per_block) {
     const double angle = (static_cast<double>(pos[r]) / factor) * inv_freq;
