@@ -39,14 +39,21 @@
  *     device memory and never frees what it is given.
  *   - All work is enqueued on `cuda_stream` (a cudaStream_t; NULL = legacy
  *     default stream) and the call returns without synchronising.  Stream
- *     order is kept: the decode kernels launch as programmatic dependents of
- *     the preceding grid (their blocks may become resident early) but wait on
- *     the device for it to finish before they read or write any memory.  The
+ *     order is kept: the decode kernels and the RoPE table kernel launch as
+ *     programmatic dependents of the preceding grid (their blocks may become
+ *     resident early) but wait on the device for it to finish before they
+ *     read or write any memory.  The
  *     decode combine and the RoPE table kernels allow their own programmatic
  *     dependents to launch early; a caller kernel launched with the
  *     programmatic-serialization attribute after them must wait
  *     (griddepcontrol.wait / cudaGridDependencySynchronize) before reading
  *     their outputs, as for any such launch.
+ *   - cos/sin rows are LLaMA RoPE table rows: the second half of a row repeats
+ *     the first (columns i and i + head_dim/2 hold the same value, because the
+ *     table concatenates the frequencies with themselves), as llama_rope_table
+ *     writes them.  Kernels may read either copy (the bf16 prefill kernel
+ *     reads only the first half); rows whose halves differ are not supported
+ *     and are not detected.
  *   - `dtype` (llama_dtype) applies to q, k, v, the caches and out together.
  *     LLAMA_DT_BF16 runs the tensor-core kernels (tcgen05 prefill, mma decode)
  *     with fp32 accumulation and an fp32 softmax; the probabilities are

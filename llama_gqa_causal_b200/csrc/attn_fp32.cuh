@@ -113,24 +113,49 @@ __global__ void __launch_bounds__(128) attn_fp32_kernel(Fp32Params p) {
 
   for (int j0 = 0; j0 < n_keys; j0 += KT) {
     __syncthreads();
-    // ---- stage K (rotated) and V for keys [j0, j0 + KT)
-    for (int idx = tid; idx < KT * D; idx += 128) {
-      const int j = idx / D, d = idx - (idx / D) * D;
-      const int key = j0 + j;
-      float kx = 0.f, vx = 0.f;
-      if (key < n_keys) {
-        const float* kr = kbase + key * kv_row_stride;
-        kx = kr[d];
-        if (rotate_k) {
-          const float* cr = p.cos + (static_cast<size_t>(b) * p.S + key) * D;
-          const float* sr = p.sin + (static_cast<size_t>(b) * p.S + key) * D;
-          const float rot = (d < D / 2) ? -kr[d + D / 2] : kr[d - D / 2];
-          kx = fmaf(kx, cr[d], rot * sr[d]);
+    // ---- stage K (rotated) and V for keys [j0, j0 + KT).  128 is a multiple
+    // of D, so a thread keeps one column d and takes every (128 / D)-th key;
+    // the global loads of a batch of keys are all issued before any of them is
+    // used, so a tile costs a few memory round trips rather than one per key.
+    {
+      constexpr int PER = KT * D / 128;  // tile elements per thread
+      constexpr int BATCH = 8;
+      constexpr int JSTEP = 128 / D;
+      static_assert(128 % D == 0 && PER % BATCH == 0, "staging layout");
+      const int d = tid % D, j_first = tid / D;
+      const int dp = (d < D / 2) ? d + D / 2 : d - D / 2;  // rotation partner of d
+      const bool lower = d < D / 2;
+#pragma unroll 1
+      for (int i0 = 0; i0 < PER; i0 += BATCH) {
+        float kx[BATCH], kp[BATCH], cr[BATCH], sr[BATCH], vx[BATCH];
+#pragma unroll
+        for (int u = 0; u < BATCH; ++u) {
+          const int key = j0 + j_first + (i0 + u) * JSTEP;
+          kx[u] = kp[u] = cr[u] = sr[u] = vx[u] = 0.f;
+          if (key < n_keys) {
+            const float* kr = kbase + key * kv_row_stride;
+            kx[u] = kr[d];
+            vx[u] = vbase[key * kv_row_stride + d];
+            if (rotate_k) {
+              const size_t t = (static_cast<size_t>(b) * p.S + key) * D + d;
+              kp[u] = kr[dp];
+              cr[u] = p.cos[t];
+              sr[u] = p.sin[t];
+            }
+          }
         }
-        vx = vbase[key * kv_row_stride + d];
+#pragma unroll
+        for (int u = 0; u < BATCH; ++u) {
+          const int j = j_first + (i0 + u) * JSTEP;
+          float k_out = kx[u];
+          if (rotate_k) {
+            const float rot = lower ? -kp[u] : kp[u];
+            k_out = fmaf(kx[u], cr[u], rot * sr[u]);
+          }
+          ks[j][d] = k_out;
+          vs[j][d] = vx[u];
+        }
       }
-      ks[j][d] = kx;
-      vs[j][d] = vx;
     }
     __syncthreads();
 

@@ -369,6 +369,7 @@ int decode_bf16(const void* q, const void* kc, const void* vc, const int* lens, 
   }
   if (se != cudaSuccess) {
     fprintf(stderr, "llama_attn: decode launch failed: %s\n", cudaGetErrorString(se));
+    (void)cudaGetLastError();  // reported here, not again by a later call
     return LLAMA_ERR_CUDA;
   }
   if (int e = launch_status()) return e;
@@ -388,6 +389,7 @@ int decode_bf16(const void* q, const void* kc, const void* vc, const int* lens, 
                                            prefix, o, bsz, H, Hkv, group, hchunks, n_ctas);
   if (e != cudaSuccess) {
     fprintf(stderr, "llama_attn: combine launch failed: %s\n", cudaGetErrorString(e));
+    (void)cudaGetLastError();  // reported here, not again by a later call
     return LLAMA_ERR_CUDA;
   }
   return launch_status();
@@ -468,8 +470,24 @@ int llama_rope_table(const long long* pos, int bsz, int seq, int head_dim, doubl
   if (half <= la::kRopeHostFreqs)
     for (int i = 0; i < half; ++i)
       freqs.inv[i] = std::exp(-(2.0 * i / head_dim) * std::log(theta));
-  la::rope_table_kernel<<<blocks, threads, 0, as_stream(cuda_stream)>>>(
-      pos, n, head_dim, theta, pos_scale_factor, cos, sin, freqs);
+  // launched as a programmatic dependent of the preceding grid: the launch
+  // overlaps that grid's drain, and the kernel waits for it on the device
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(blocks);
+  cfg.blockDim = dim3(threads);
+  cfg.stream = as_stream(cuda_stream);
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, la::rope_table_kernel, pos, n, head_dim, theta,
+                                           pos_scale_factor, cos, sin, freqs);
+  if (e != cudaSuccess) {
+    fprintf(stderr, "llama_attn: rope table launch failed: %s\n", cudaGetErrorString(e));
+    (void)cudaGetLastError();  // reported here, not again by a later call
+    return LLAMA_ERR_CUDA;
+  }
   return launch_status();
 }
 

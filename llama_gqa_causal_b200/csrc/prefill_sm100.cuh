@@ -418,16 +418,17 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
       // Warp-cooperative: per step a warp takes 32 / (D/4) rows, each lane one
       // bf16 pair (d, d+1) of the first half and its partner pair d + D/2, with
       // coalesced cos/sin loads; 32 lanes cover whole 128-byte rows, so the
-      // swizzled accesses are free of bank conflicts.  The cos/sin values of
-      // half the warp's rows are loaded into registers at once (the first half
-      // while the Q copy is still in flight), so the table reads cost two
-      // round trips rather than one per row.
+      // swizzled accesses are free of bank conflicts.  A LLaMA cos/sin row
+      // repeats its first half (the frequencies are concatenated with
+      // themselves), so columns d and d + D/2 share one value and only the
+      // first half is read.  The values of all the warp's rows are loaded into
+      // registers at once, while the Q copy is still in flight: the table
+      // reads cost one round trip.
       {
         if (p.cos != nullptr) {
           constexpr int PAIRS = D / 4;             // bf16 pairs in half a row
           constexpr int ROWS_PER_STEP = 32 / PAIRS;
           constexpr int STEPS = 32 / ROWS_PER_STEP;  // steps covering the warp's 32 rows
-          constexpr int BATCH = STEPS / 2;
           uint8_t* qs = reinterpret_cast<uint8_t*>(&s.q[t][0]);
           const int wq = warp & 3;                 // warp index inside the warpgroup
           const int pr = lane % PAIRS, rsub = lane / PAIRS;
@@ -435,38 +436,31 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
           const int d2 = d + D / 2;                // its rotation partner
           const uint32_t colb = static_cast<uint32_t>((d % 64) / 8), inb = (d % 8) * 2;
           const uint32_t colb2 = static_cast<uint32_t>((d2 % 64) / 8);
-          bool q_ok = true;
+          float2 cf[STEPS], sf[STEPS];
 #pragma unroll
-          for (int bt = 0; bt < 2; ++bt) {
-            float2 c1[BATCH], c2[BATCH], s1[BATCH], s2[BATCH];
+          for (int st = 0; st < STEPS; ++st) {
+            const int rr = wq * 32 + st * ROWS_PER_STEP + rsub;
+            // rows past S_b are discarded (zeros, padding or the next packed
+            // sequence); any of this entry's table rows serves them
+            const int pos = min(my_pb * BM + rr, S_b - 1);
+            const size_t trow = ((VARLEN == 2 ? static_cast<size_t>(tok0)
+                                               : static_cast<size_t>(b) * p.S) + pos) * D;
+            cf[st] = *reinterpret_cast<const float2*>(p.cos + trow + d);
+            sf[st] = *reinterpret_cast<const float2*>(p.sin + trow + d);
+          }
+          if (mbar_wait(&s.q_loaded[t], 0)) {
 #pragma unroll
-            for (int st = 0; st < BATCH; ++st) {
-              const int rr = wq * 32 + (bt * BATCH + st) * ROWS_PER_STEP + rsub;
-              // rows past S_b are discarded (zeros, padding or the next packed
-              // sequence); any of this entry's table rows serves them
-              const int pos = min(my_pb * BM + rr, S_b - 1);
-              const size_t trow = ((VARLEN == 2 ? static_cast<size_t>(tok0)
-                                                 : static_cast<size_t>(b) * p.S) + pos) * D;
-              c1[st] = *reinterpret_cast<const float2*>(p.cos + trow + d);
-              c2[st] = *reinterpret_cast<const float2*>(p.cos + trow + d2);
-              s1[st] = *reinterpret_cast<const float2*>(p.sin + trow + d);
-              s2[st] = *reinterpret_cast<const float2*>(p.sin + trow + d2);
-            }
-            if (bt == 0) q_ok = mbar_wait(&s.q_loaded[t], 0);
-            if (q_ok) {
-#pragma unroll
-              for (int st = 0; st < BATCH; ++st) {
-                const int rr = wq * 32 + (bt * BATCH + st) * ROWS_PER_STEP + rsub;
-                const uint32_t row = static_cast<uint32_t>(rr) * 128;
-                uint32_t* p1 = reinterpret_cast<uint32_t*>(qs + (d / 64) * BLOCK_BYTES + row +
-                                                           (((colb ^ (rr & 7)) << 4) | inb));
-                uint32_t* p2 = reinterpret_cast<uint32_t*>(qs + (d2 / 64) * BLOCK_BYTES + row +
-                                                           (((colb2 ^ (rr & 7)) << 4) | inb));
-                const uint32_t xa = *p1, za = *p2;
-                const float x0 = bf16lo(xa), x1 = bf16hi(xa), z0 = bf16lo(za), z1 = bf16hi(za);
-                *p1 = pack_bf16x2(fmaf(x0, c1[st].x, -z0 * s1[st].x), fmaf(x1, c1[st].y, -z1 * s1[st].y));
-                *p2 = pack_bf16x2(fmaf(z0, c2[st].x, x0 * s2[st].x), fmaf(z1, c2[st].y, x1 * s2[st].y));
-              }
+            for (int st = 0; st < STEPS; ++st) {
+              const int rr = wq * 32 + st * ROWS_PER_STEP + rsub;
+              const uint32_t row = static_cast<uint32_t>(rr) * 128;
+              uint32_t* p1 = reinterpret_cast<uint32_t*>(qs + (d / 64) * BLOCK_BYTES + row +
+                                                         (((colb ^ (rr & 7)) << 4) | inb));
+              uint32_t* p2 = reinterpret_cast<uint32_t*>(qs + (d2 / 64) * BLOCK_BYTES + row +
+                                                         (((colb2 ^ (rr & 7)) << 4) | inb));
+              const uint32_t xa = *p1, za = *p2;
+              const float x0 = bf16lo(xa), x1 = bf16hi(xa), z0 = bf16lo(za), z1 = bf16hi(za);
+              *p1 = pack_bf16x2(fmaf(x0, cf[st].x, -z0 * sf[st].x), fmaf(x1, cf[st].y, -z1 * sf[st].y));
+              *p2 = pack_bf16x2(fmaf(z0, cf[st].x, x0 * sf[st].x), fmaf(z1, cf[st].y, x1 * sf[st].y));
             }
           }
           fence_proxy_async_smem();

@@ -32,6 +32,10 @@ __global__ void rope_table_kernel(const long long* __restrict__ pos, long long n
   // a programmatic dependent launched after this kernel (a decode reading the
   // table) may be scheduled now; it waits for this grid to finish
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  // this kernel is itself launched as a programmatic dependent of whatever
+  // precedes it: the positions (and the table's own storage) are touched only
+  // once that grid has finished
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const int half = D / 2;
   const int i = static_cast<int>(threadIdx.x % half);
   const int rows_per_block = static_cast<int>(blockDim.x / half);
