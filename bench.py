@@ -461,11 +461,41 @@ def _decode_phase(args, ws, local, dev, stream, line):
     d1.record(stream)
     torch.cuda.synchronize()
     _barrier(ws)
-    for i in range(dsteps):
-        decode_step(i, devs[i])
-    torch.cuda.synchronize()
+    # the decode call alone (roofline figure).  Events between direct launches
+    # would also time the split kernel's launch, which the call otherwise
+    # overlaps with the previous grid, so with graphs the call (split +
+    # combine, tables formed beforehand) is replayed as a graph of its own and
+    # the train's mean is taken; without graphs, events go around each call.
+    tabs = [api.rope_table(d["qpos"].view(-1, 1), dcfg.head_dim, dcfg.theta, dcfg.factor)
+            for d in insts]
+
+    def decode_call(i):
+        d = insts[i % 2]
+        cos, sin = tabs[i % 2]
+        api.decode(d["q"], d["k_cache"], d["v_cache"], d["lens"], cos.view(dcfg.bsz, -1),
+                   sin.view(dcfg.bsz, -1), scale=dcfg.scale, out=dout, workspace=dws)
+
+    call_graphs = None if graphs is None else [_capture(lambda i=i: decode_call(i)) for i in range(2)]
+    if call_graphs is not None and all(g_ is not None for g_ in call_graphs):
+        for i in range(max(args.warmup, 3)):
+            call_graphs[i % 2].replay()
+        torch.cuda.synchronize()
+        c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        c0.record(stream)
+        for i in range(dsteps):
+            call_graphs[i % 2].replay()
+        c1.record(stream)
+        torch.cuda.synchronize()
+        ms_dec_call = _max_over_ranks(c0.elapsed_time(c1) / dsteps, ws)
+        call_timing = "graph replays of the call alone (train mean)"
+    else:
+        for i in range(dsteps):
+            decode_step(i, devs[i])
+        torch.cuda.synchronize()
+        ms_dec_call = _max_over_ranks(statistics.mean(a.elapsed_time(b) for a, b in devs), ws)
+        call_timing = "events around each direct call"
+    del call_graphs
     ms_dec_total = _max_over_ranks(d0.elapsed_time(d1), ws)
-    ms_dec_call = _max_over_ranks(statistics.mean(a.elapsed_time(b) for a, b in devs), ws)
     dec_value = replicas.job_throughput(dbytes, dsteps, ms_dec_total, ws) / 1e9
     dec_achieved = dbytes / (ms_dec_call * 1e-3) / 1e9
     assert api.device_status() == api.LLAMA_OK
@@ -521,6 +551,7 @@ def _decode_phase(args, ws, local, dev, stream, line):
         "roofline": {
             "bound": "hbm",
             "kernel": "llama_attn_decode (decode_bf16_kernel + decode_combine_kernel)",
+            "timing": call_timing,
             "achieved": round(dec_achieved, 1),
             "peak": hbm,
             "unit": "GB/s",
@@ -644,7 +675,9 @@ def run_reference(args, rank, ws):
 
 
 def run_configs(args):
-    """One JSON line per named workload: mean duration of the library call."""
+    """One JSON line per named workload: mean device time of the library call
+    (a train of CUDA-graph replays of the call; events around each direct call
+    with --no-graph)."""
     from llama_gqa_causal_b200 import api
     api.load()
     dev = torch.device("cuda", 0)
@@ -654,9 +687,27 @@ def run_configs(args):
     steps = max(args.steps, 1)
 
     def timed(call):
+        """Mean device time of one call: the call captured as a CUDA graph and
+        replayed `steps` times between two events (so that the binding's host
+        work, which exceeds the small workloads' kernel time, is not what is
+        timed); events around each direct call where capture is not possible."""
         for _ in range(args.warmup):
             call()
         torch.cuda.synchronize()
+        graph = None if args.no_graph else _capture(call)
+        if graph is not None:
+            for _ in range(args.warmup):
+                graph.replay()
+            torch.cuda.synchronize()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            for _ in range(steps):
+                graph.replay()
+            b.record(stream)
+            torch.cuda.synchronize()
+            assert api.device_status() == api.LLAMA_OK
+            del graph
+            return a.elapsed_time(b) / steps
         evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
                for _ in range(steps)]
         for a, b in evs:
