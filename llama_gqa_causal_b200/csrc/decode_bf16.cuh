@@ -224,7 +224,19 @@ __global__ void __launch_bounds__(dec::THREADS, 1) decode_bf16_kernel(
   if (x0 >= x1) return;  // uniform across the CTA: no share
 
   if (warp == NCW) {  // ---------------------------------------------- TMA producer
+    // batch entry of the share's first chunk: the largest b with
+    // chunk_prefix[b] * per_b <= x0, by binary search (a scan from entry 0
+    // would delay the first copies of the last CTAs by up to bsz steps of
+    // dependent shared-memory loads)
     int b = 0;
+    {
+      int hi = p.bsz - 1;
+      while (b < hi) {
+        const int mid = (b + hi + 1) >> 1;
+        if (static_cast<long long>(s.chunk_prefix[mid]) * per_b <= x0) b = mid;
+        else hi = mid - 1;
+      }
+    }
     int it = 0;  // tiles issued
     bool ok = true;
     bool home = false;
