@@ -6,6 +6,11 @@ torch when the caller does not pass them, and a non-zero status raises.  Every
 step of the computation runs in the library's kernels.  There is no CPU
 fallback: without the built library, or on a tensor that is not on a CUDA
 device, the call raises.
+
+cos/sin arguments are LLaMA RoPE tables as ``rope_table`` returns them: the
+second half of every row repeats the first (the frequencies concatenated with
+themselves).  The kernels may read either copy; a table whose halves differ
+is not supported (include/llama_attn.h states the same for the C ABI).
 """
 from __future__ import annotations
 
