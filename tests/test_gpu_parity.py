@@ -84,6 +84,17 @@ def test_rope_table_ntk_matches_oracle(D, alpha):
     assert np.abs(sin[0].cpu().double().numpy() - s).max() < 2e-7
 
 
+@pytest.mark.parametrize("D", [64, 128])
+def test_rope_tables_repeat_their_first_half(D):
+    # the prefill kernel reads only the first half of each row, which the
+    # header requires to repeat in the second: both table entry points write
+    # the two halves bit for bit alike
+    pos = torch.randint(0, 1 << 20, (2, 300), generator=torch.Generator().manual_seed(3)).cuda()
+    for cos, sin in (api.rope_table(pos, D, 10000.0, 2.0), api.rope_table_ntk(pos, D, 10000.0, 4.0)):
+        assert torch.equal(cos[..., :D // 2], cos[..., D // 2:])
+        assert torch.equal(sin[..., :D // 2], sin[..., D // 2:])
+
+
 # ----------------------------------------------------------------------------- named workloads
 
 def test_tiny_fp32_workload():
