@@ -324,22 +324,23 @@ __device__ __forceinline__ void fadd2(float& d0, float& d1, float a0, float a1, 
 }
 // 2^x for a pair of finite values on the FMA and integer pipes instead of the
 // MUFU unit.  Range reduction: adding 1.5*2^23 rounds x to the integer n held
-// in the low mantissa bits of t; f = x - n lies in [-1/2, 1/2]; 2^f is a cubic
-// whose coefficients minimise the maximum relative error on that interval
-// (7.5e-5; fitted by csrc/fit_exp2_poly.py); n is then added to the exponent
-// field.  Inputs below -127 are clamped (the result is then < 2^-126).
+// in the low mantissa bits of t; f = x - n lies in [-1/2, 1/2]; 2^f is a
+// quadratic whose coefficients minimise the maximum relative error on that
+// interval (1.7e-3, fitted by csrc/fit_exp2_poly.py: below the 2^-8 relative
+// step of the bf16 rounding the probabilities go through, and the same value
+// enters both P and the row sum); n is then added to the exponent field.
+// Inputs below -127 are clamped (the result is then < 2^-126).
 __device__ __forceinline__ void exp2_poly2(float& y0, float& y1, float x0, float x1) {
   constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
-  constexpr float c0 = 0.9999280571937561f, c1 = 0.6932609677314758f;
-  constexpr float c2 = 0.2426111251115799f, c3 = 0.0551716685295105f;
+  constexpr float c0 = 1.0004431009292603f, c1 = 0.7034479975700378f;
+  constexpr float c2 = 0.23842893540859222f;
   x0 = fmaxf(x0, -127.f);
   x1 = fmaxf(x1, -127.f);
   float t0, t1, n0, n1, f0, f1, q0, q1;
   fadd2(t0, t1, x0, x1, kRound, kRound);      // round(x) in the low bits of t
   fadd2(n0, n1, t0, t1, -kRound, -kRound);    // n = round(x) as a float
   ffma2(f0, f1, n0, n1, -1.f, -1.f, x0, x1);  // f = x - n
-  ffma2(q0, q1, c3, c3, f0, f1, c2, c2);
-  ffma2(q0, q1, q0, q1, f0, f1, c1, c1);
+  ffma2(q0, q1, c2, c2, f0, f1, c1, c1);
   ffma2(q0, q1, q0, q1, f0, f1, c0, c0);
   y0 = __int_as_float(__float_as_int(q0) + (__float_as_int(t0) << 23));
   y1 = __int_as_float(__float_as_int(q1) + (__float_as_int(t1) << 23));
