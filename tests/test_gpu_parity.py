@@ -307,3 +307,33 @@ def test_repeated_runs_are_bitwise_identical():
     d2 = api.decode(*args)
     torch.cuda.synchronize()
     assert torch.equal(d1, d2)
+
+
+def test_decode_over_more_caches_than_the_tensor_map_memo_holds():
+    # the library memoises 32 encoded tensor maps (a map is a pure function of
+    # base address, dimensions, strides and box); 20 cache pairs need 40, so
+    # the second pass, in reverse order, runs on maps evicted and encoded again
+    dev = torch.device("cuda")
+    b, H, Hkv, D, L = 2, 8, 2, 64, 200
+    cases = []
+    for i in range(20):
+        cfg, x = W.small_decode(b, H, Hkv, D, L, torch.bfloat16, seed=500 + i)
+        cos, sin = api.rope_table(x["qpos"].view(-1, 1).to(dev), D, cfg.theta, cfg.factor)
+        cases.append((cfg, x, {n: x[n].to(dev) for n in ("q", "k_cache", "v_cache", "lens")},
+                      cos.view(b, D), sin.view(b, D)))
+
+    def run(case):
+        cfg, _, d, cos, sin = case
+        return api.decode(d["q"], d["k_cache"], d["v_cache"], d["lens"], cos, sin, scale=cfg.scale)
+
+    first = [run(c) for c in cases]
+    again = [run(c) for c in reversed(cases)][::-1]
+    torch.cuda.synchronize()
+    assert api.device_status() == api.LLAMA_OK
+    for o1, o2 in zip(first, again):
+        assert torch.equal(o1, o2)
+    for i in (0, 19):
+        cfg, x = cases[i][0], cases[i][1]
+        ref = oracle.decode(x["q"], x["k_cache"], x["v_cache"], x["lens"], x["qpos"],
+                            theta=cfg.theta, factor=cfg.factor, scale=cfg.scale)
+        _check(first[i], ref, torch.bfloat16, f"memo case {i}")
