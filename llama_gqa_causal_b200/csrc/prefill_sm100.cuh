@@ -61,10 +61,18 @@ constexpr int NQ = 2;         // Q tiles (units) per CTA
 constexpr int KSTAGES = LA_PF_KSTAGES;  // K tile ring depth
 constexpr int VSTAGES = LA_PF_VSTAGES;  // V tile ring depth
 constexpr int THREADS = 384;  // warpgroup 0: TMA + MMA warps; warpgroups 1, 2: softmax
-// Register budget per warpgroup after setmaxnreg: each SMSP holds one warp of
-// every warpgroup, 56 + 224 + 224 registers x 32 lanes = 16128 <= 16384.
+// Register budget per warpgroup after setmaxnreg.  setmaxnreg.inc can only
+// take registers that the block was launched with: 384 threads x 168 (the
+// most __launch_bounds__(384, 1) allows), i.e. 504 per lane over the three
+// warpgroups that share an SMSP: 56 + 224 + 224.  A split above that makes the
+// increasing warps wait for registers that never come free, so it is refused
+// here.
 constexpr int kRegsControl = 56;
 constexpr int kRegsSoftmax = 224;
+constexpr int kRegsAtLaunch = (65536 / THREADS) / 8 * 8;  // 168
+static_assert(kRegsControl % 8 == 0 && kRegsSoftmax % 8 == 0, "setmaxnreg takes multiples of 8");
+static_assert(kRegsControl + 2 * kRegsSoftmax <= 3 * kRegsAtLaunch,
+              "setmaxnreg split exceeds the registers the block is launched with");
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 // Of every 8 consecutive pairs of probabilities in an interior tile, this
 // many are exponentiated on the FMA pipe (exp2_poly2), the rest on MUFU.
